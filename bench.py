@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon optimizer step on one B200 per process.
+
+A step is the whole hot path over one batch of matrices: momentum + Nesterov +
+Frobenius norm + cast (1 kernel), then 10 hybrid Newton-Schulz steps (3 grouped
+GEMM kernels each), the last one fused with the RMS rescale, decoupled weight
+decay and parameter update. Default workload: 64 square 1024 x 1024 fp32
+matrices (W, G, M resident in HBM, 805 MB, larger than the 126 MB L2, so no
+explicit L2 flush between steps), bf16 Newton-Schulz operands.
+
+Metric: Newton-Schulz TFLOP/s of the whole step, with the FLOPs the metric
+defines, 10 (4 r^2 c + 2 r^3) per matrix (r = min(n, m), c = max(n, m)), and
+the step time in ms. Multi-GPU: every rank runs its own batch (independent
+problems, no data-path collective, weak scaling); value = FLOPs of all ranks /
+the slowest rank's time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference     # the float64 CPU oracle, timed on a sample
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon step ms & Newton–Schulz TFLOPS (% of B200 bf16 dense peak) per shape set"
+UNIT = "TFLOP/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="batch64_1024")
+    ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
+    return ap.parse_args()
+
+
+def metric_flops(shapes, ns_steps=10):
+    """FLOPs the metric defines: ns_steps * (4 r^2 c + 2 r^3) per matrix."""
+    tot = 0.0
+    for n, m in shapes:
+        r, c = min(n, m), max(n, m)
+        tot += ns_steps * (4.0 * r * r * c + 2.0 * r ** 3)
+    return tot
+
+
+def apply_bytes(shapes):
+    """Algorithmic HBM bytes of one Apply launch: B (bf16 r x r) and X (bf16
+    r x c) operands read once, fp32 iterate read and written, bf16 iterate
+    written: 2 r^2 + 12 r c per matrix."""
+    return sum(2.0 * min(n, m) ** 2 + 12.0 * min(n, m) * max(n, m) for n, m in shapes)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_rate(wl_cpu_mats, hyper, budget_s=None):
+    """Time the float64 oracle (as it stands) on a list of (W, G, M) numpy
+    matrices; returns (TFLOP/s by the metric's count, seconds, matrices done)."""
+    from oracle import muon_oracle
+
+    t0 = time.perf_counter()
+    done = []
+    for W, G, M in wl_cpu_mats:
+        muon_oracle.muon_step(W, G, M, lr=hyper["lr"], mu=hyper["mu"], wd=hyper["wd"],
+                              gamma=hyper["gamma"], nesterov_on=hyper["nesterov"])
+        done.append(W.shape)
+        if budget_s is not None and time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return metric_flops(done) / dt / 1e12, dt, len(done)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = [l.split(",") for l in open(self.path).read().splitlines() if l.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_from_profile(config):
+    """Per-launch DRAM bytes of the Apply kernel from the committed ncu summary
+    (null if there is none for this workload)."""
+    path = os.path.join(ROOT, "profiles", f"ns_apply_{config}.md")
+    if not os.path.exists(path):
+        return None
+    m = re.search(r"^traffic_per_launch_bytes:\s*([0-9.eE+]+)\s*$", open(path).read(), re.M)
+    return float(m.group(1)) if m else None
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the float64 CPU oracle, timed on host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import numpy as np
+    import workloads
+
+    # a bounded sample of the workload: one matrix of its first shape per step
+    wl = workloads.make(args.config, device="cpu", **_small_kwargs(args.config))
+    mats = [(wl.W[k].double().numpy(), wl.G[k].double().numpy(), wl.M[k].double().numpy())
+            for k in range(1)]
+    h = wl.hyper
+    for _ in range(args.warmup):
+        cpu_oracle_rate(mats, h)
+    times = []
+    for _ in range(args.steps):
+        rate, dt, _n = cpu_oracle_rate(mats, h)
+        times.append(dt)
+    tot = sum(times)
+    value = metric_flops([mats[0][0].shape]) * args.steps / tot / 1e12
+    cores = oracle_threads()
+    sample = f"1 matrix {mats[0][0].shape[0]}x{mats[0][0].shape[1]} of {args.config} per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.config},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _small_kwargs(config):
+    # the reference arm needs only one matrix of the workload's shape
+    if config == "batch64_1024":
+        return {"count": 1}
+    if config == "dense_d4096":
+        return {"layers": 1}
+    if config == "moe_64x3":
+        return {"experts": 1}
+    if config.startswith("sweep_"):
+        return {"count": 1}
+    return {}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import muon_step_b200 as ms
+    import workloads
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs CUDA GPUs")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = workloads.make(args.config, device=dev)
+    h = wl.hyper
+    params = [(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)]
+    plan = ms.MuonPlan(params, precision=args.precision)
+    ws = plan.alloc_workspace()
+    kinds = plan.launches()
+    ns_steps = (len(kinds) - 1) // 3
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan.execute(ws, lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"], gamma=h["gamma"],
+                     nesterov=h["nesterov"], stream=stream)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+
+    # ---- timed region: device time with events, per-launch events inside
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(kinds))]
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for k in range(args.steps):
+        plan.set_events(ev[k])
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    plan.set_events(None)
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    status = ms.sync_status()
+    if status != 0:
+        raise SystemExit(f"device error status {status}")
+
+    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    flops_rank = metric_flops(wl.shapes, ns_steps)
+    value = flops_rank * world * args.steps / (ms_max / 1e3) / 1e12
+
+    # per-kernel durations over the timed region
+    per_kind = {}
+    for k in range(args.steps):
+        for i, kd in enumerate(kinds):
+            per_kind.setdefault(kd, []).append(ev[k][2 * i].elapsed_time(ev[k][2 * i + 1]))
+    avg = {kd: sum(v) / len(v) for kd, v in per_kind.items()}
+    share = {kd: sum(v) for kd, v in per_kind.items()}
+    tot_kernel = sum(share.values())
+
+    peaks, peak_src = load_peaks()
+    g_fl, p_fl, a_fl = plan.flops()
+    apply_flops = a_fl / ns_steps
+    apply_b = apply_bytes(wl.shapes)
+    apply_ms = avg.get(3, float("nan"))
+    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    hbm_peak = float(peaks["hbm_gbs"])
+    t_tensor = apply_flops / (tensor_peak * 1e12)
+    t_hbm = apply_b / (hbm_peak * 1e9)
+    traffic = traffic_from_profile(args.config)
+    if t_hbm >= t_tensor:
+        achieved = apply_b / (apply_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic}
+    else:
+        achieved = apply_flops / (apply_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "traffic": traffic}
+    roof["kernel"] = "stage_tc_kernel<Apply>" if args.precision == "bf16" else "stage_simt_kernel<Apply>"
+    roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'HBM copy'})"
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        G_dev = [grp[1] for grp in wl.groups.values()]
+        W_dev = [grp[0] for grp in wl.groups.values()]
+        G_host = [g.cpu().pin_memory() for g in G_dev]
+        W_host = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in W_dev]
+        h2d = sum(g.numel() * 4 for g in G_host)
+        d2h = sum(w.numel() * 4 for w in W_host)
+        for _ in range(2):
+            for gh, gd in zip(G_host, G_dev):
+                gd.copy_(gh, non_blocking=True)
+            step()
+            for wh, wd in zip(W_host, W_dev):
+                wh.copy_(wd, non_blocking=True)
+        torch.cuda.synchronize()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e_s.record(stream)
+        for _ in range(args.steps):
+            for gh, gd in zip(G_host, G_dev):
+                gd.copy_(gh, non_blocking=True)
+            step()
+            for wh, wd in zip(W_host, W_dev):
+                wh.copy_(wd, non_blocking=True)
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([e_s.elapsed_time(e_e)], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": flops_rank * world * args.steps / (float(te.item()) / 1e3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": float(te.item()) / args.steps}
+        assert ms.sync_status() == 0
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ks = list(range(min(args.cpu_sample, wl.count)))
+        mats = [(wl.W[k].double().cpu().numpy(), wl.G[k].double().cpu().numpy(),
+                 wl.M[k].double().cpu().numpy()) for k in ks]
+        rate, dt, done = cpu_oracle_rate(mats, h, budget_s=30.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{done} of {wl.count} matrices of {args.config}, {dt:.1f} s of float64 numpy"}
+
+    if rank == 0:
+        names = {0: "elementwise", 1: "gram", 2: "poly", 3: "apply", 4: "apply_update"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": args.precision,
+            "data": "synthetic",
+            "config": {"workload": args.config, "matrices": wl.count,
+                       "shapes": sorted({f"{n}x{m}" for n, m in wl.shapes}),
+                       "ns_steps": ns_steps, "precision": args.precision,
+                       "l2": "inputs larger than L2 (no flush)" if wl.elements() * 12 > 126e6
+                             else "inputs smaller than L2",
+                       "metric_flops_per_step": flops_rank},
+            "pct_of_peak": {"bf16_burst": value / float(peaks.get("bf16_tflops", 1590.0)),
+                            "bf16_sustained": value / tensor_peak},
+            "roofline": roof,
+            "kernels_ms_avg": {names[k]: v for k, v in sorted(avg.items())},
+            "kernels_share": {names[k]: v / tot_kernel for k, v in sorted(share.items())},
+            "executed_tflops": (g_fl + p_fl + a_fl) / (ms_per_step / 1e3) / 1e12,
+            "gpu_launches": len(kinds) * args.steps,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del plan
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * muon_step.h - C ABI of the B200 (sm_100a) Muon optimizer step library.
+ *
+ * The method (sources cited by page title and section):
+ *
+ *   [V4-breakdown] "Muon 优化器完全拆解：矩阵级正交化更新如何撑起万亿 MoE 训练",
+ *                  section "V4 的完整更新公式，逐行拆解", Algorithm 1
+ *                  "Muon Optimizer for DeepSeek-V4" and its five steps.
+ *   [V4-book]      "Ch 06 · Muon — 矩阵参数的指南针" (DeepSeek-V4-book ch. 6),
+ *                  §3 (Newton-Schulz), §4 (hybrid 8 + 2 schedule),
+ *                  §5 Algorithm 1 "Muon Optimizer (V4 Hybrid)".
+ *
+ * For every 2-D weight W (n x m) with gradient G and momentum buffer M:
+ *
+ *   M   <- mu M + G                                  momentum
+ *   N    = mu M + G        (M itself if nesterov=0)  Nesterov look-ahead
+ *   X    = N / (||N||_F + eps), transposed when n > m (rows <= cols)
+ *   X   <- a_k X + b_k (X X^T) X + c_k (X X^T)^2 X   k = 1 .. steps
+ *   O'   = X, transposed back                       (orthogonalised direction)
+ *   W   <- W (1 - lr wd) - lr gamma sqrt(max(n, m)) O'
+ *
+ * The default schedule is 8 steps of (3.4445, -4.7750, 2.0315) then 2 steps
+ * of (2, -1.5, 0.5), with eps = 1e-7.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are caller-owned, contiguous, row-major fp32 DEVICE arrays.
+ *     Distinct matrices must not overlap. The library allocates no device
+ *     memory: all scratch lives in the caller's workspace.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All device work is asynchronous on that stream; nothing
+ *     synchronises except muon_sync_status().
+ *   - Argument errors are reported synchronously and leave the device
+ *     untouched. Device-side failures (a bounded wait that expired) set a
+ *     per-device error word that muon_sync_status() reports and clears.
+ *   - NaN / Inf in the inputs are not checked; they propagate as in the
+ *     plain definition.
+ */
+#ifndef MUON_STEP_H
+#define MUON_STEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUON_ABI_VERSION 1
+#define MUON_MAX_NS_STEPS 64
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, bad count, bad schedule */
+  MUON_ERR_WORKSPACE = 2,   /* workspace NULL, misaligned (256 B) or too small */
+  MUON_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  MUON_ERR_UNSUPPORTED = 4, /* no sm_100 device, or a size beyond the limits */
+  MUON_ERR_TIMEOUT = 5      /* a device-side bounded wait expired */
+} muon_status_t;
+
+/* Newton-Schulz operand precision. BF16: bf16 tensor-core operands with fp32
+ * accumulation and an fp32 master copy of the iterate. FP32: fp32 operands on
+ * the CUDA cores (validation; slow). Momentum and update are fp32 in both. */
+typedef enum { MUON_NS_BF16 = 0, MUON_NS_FP32 = 1 } muon_precision_t;
+
+/* One matrix of a Muon step ([V4-breakdown] Algorithm 1 inputs). */
+typedef struct {
+  float* W;       /* n x m weight, updated in place */
+  const float* G; /* n x m gradient, read only */
+  float* M;       /* n x m momentum buffer, updated in place */
+  float* O;       /* optional n x m output of O' (before the RMS rescale); NULL to skip */
+  int64_t n, m;   /* 1 <= n, m <= 2^31 - 1 */
+} muon_param_t;
+
+/* Newton-Schulz schedule ([V4-book] §4). `abc` is a HOST array of steps * 3
+ * floats (a, b, c per step, applied in order); 1 <= steps <= MUON_MAX_NS_STEPS;
+ * eps > 0 is added to the Frobenius norm. A NULL schedule means the hybrid
+ * 8 + 2 schedule with eps = 1e-7. The library copies it. */
+typedef struct {
+  int steps;
+  const float* abc;
+  float eps;
+} muon_ns_schedule_t;
+
+/* One matrix for ns_orthogonalize: O = O'(X) in X's orientation. */
+typedef struct {
+  const float* X; /* n x m input, read only */
+  float* O;       /* n x m output, must not overlap X */
+  int64_t n, m;
+} muon_ns_matrix_t;
+
+/* Hyper-parameters of one step ([V4-breakdown] Algorithm 1: eta, mu, lambda,
+ * gamma). nesterov != 0 selects N = mu M + G. */
+typedef struct {
+  float lr;
+  float momentum;
+  float weight_decay;
+  float gamma;
+  int nesterov;
+} muon_hyper_t;
+
+typedef struct muon_plan_s* muon_plan_t;
+
+/* ---------------------------------------------------------------- plans
+ * A plan holds, on the host, everything that depends only on the shapes:
+ * shape groups, tile lists, the workspace layout. It is built once and
+ * executed many times. Executing a plan on a workspace pointer it has not
+ * seen before first copies its descriptor tables into that workspace
+ * (cudaMemcpyAsync on `stream`); later executes on the same pointer launch
+ * kernels only, so they can be captured in a CUDA graph. Between executes the
+ * caller must not modify the workspace (or must pass another pointer). */
+
+/* Plan a Muon step over `count` matrices. Pointers in `params` are recorded
+ * and used by every execute. */
+MUON_API muon_status_t muon_plan_create(const muon_param_t* params, int count, muon_precision_t prec,
+                               const muon_ns_schedule_t* sched, muon_plan_t* plan);
+
+/* Plan ns_orthogonalize over `count` matrices. */
+MUON_API muon_status_t muon_plan_create_ns(const muon_ns_matrix_t* mats, int count,
+                                  muon_precision_t prec, const muon_ns_schedule_t* sched,
+                                  muon_plan_t* plan);
+
+/* Bytes of workspace the plan needs (device memory, 256-byte aligned). */
+MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes);
+
+/* Run the plan: one kernel for momentum / norm / cast, then three kernels per
+ * Newton-Schulz step, each one persistent launch over every matrix. `hyper` is
+ * ignored (may be NULL) for an ns_orthogonalize plan. */
+MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Number of kernel launches one execute issues, and the kind of each
+ * (0 momentum/norm/cast, 1 Gram, 2 polynomial, 3 apply, 4 apply + update). */
+MUON_API muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds);
+
+/* Optional timing: `events` holds 2 * launches cudaEvent_t (as void*); each
+ * execute records events[2k] before and events[2k + 1] after launch k on the
+ * execute's stream. count = 0 turns timing off. The caller owns the events. */
+MUON_API muon_status_t muon_plan_set_events(muon_plan_t plan, void* const* events, int count);
+
+/* Useful floating-point operations of one execute's Newton-Schulz stages, per
+ * stage kind (Gram, polynomial, apply), counted over the tiles that are
+ * actually computed and clipped to the matrices' bounds. */
+MUON_API muon_status_t muon_plan_flops(muon_plan_t plan, double* gram, double* poly, double* apply);
+
+MUON_API void muon_plan_destroy(muon_plan_t plan);
+
+/* ---------------------------------------------------------------- one-shot
+ * Plan, execute and destroy in one call. The descriptor copy is issued on
+ * `stream` from host memory that the call releases before returning (a
+ * pageable copy, staged by the CUDA runtime), so these are not meant for
+ * CUDA graph capture: capture muon_plan_execute instead. */
+
+MUON_API muon_status_t muon_workspace_size(const muon_param_t* params, int count, muon_precision_t prec,
+                                  size_t* bytes);
+
+MUON_API muon_status_t muon_step(const muon_param_t* params, int count, float lr, float momentum,
+                        float weight_decay, float gamma, int nesterov,
+                        const muon_ns_schedule_t* sched, muon_precision_t prec, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+MUON_API muon_status_t ns_workspace_size(const muon_ns_matrix_t* mats, int count, muon_precision_t prec,
+                                size_t* bytes);
+
+/* O' = HybridNewtonSchulz(X / (||X||_F + eps)) per matrix ([V4-book] §5
+ * Algorithm 1, the normalisation and the two loops), without the rescale. */
+MUON_API muon_status_t ns_orthogonalize(const muon_ns_matrix_t* mats, int count,
+                               const muon_ns_schedule_t* sched, muon_precision_t prec,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronise `stream`, then read and clear the current device's error word.
+ * Returns MUON_ERR_TIMEOUT if a bounded wait expired since the last call. */
+MUON_API muon_status_t muon_sync_status(void* stream);
+
+MUON_API const char* muon_status_string(muon_status_t status);
+
+MUON_API int muon_abi_version(void);
+
+/* Bound, in nanoseconds, on every device-side spin-wait of later launches
+ * (default 2e9). Values below 1000 are raised to 1000. */
+MUON_API void muon_set_wait_limit_ns(uint64_t ns);
+
+/* Test of the timeout path: launch one bounded wait on the device word `flag`
+ * (device memory; the wait ends when it becomes non-zero) for at most
+ * `limit_ns`. If the limit passes, the device error word gets the timeout
+ * bit, which muon_sync_status() then reports. */
+MUON_API muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_STEP_H */

@@ -1,0 +1,270 @@
+"""Python binding of the B200 Muon step library (argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels of libmuon_step.so,
+called through its C ABI (include/muon_step.h). PyTorch supplies device
+memory, the workspace and the current stream. There is no fallback: if the
+library is missing or the device is not an sm_100 GPU, calls raise.
+
+    plan = MuonPlan([(W, G, M), ...])          # fp32 CUDA tensors, n x m each
+    ws = plan.alloc_workspace()
+    plan.execute(ws, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2)
+
+    muon_step([(W, G, M)], lr=0.02)            # one-shot
+    O = ns_orthogonalize([X])                   # O' per matrix
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Iterable, Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (MUON_ERR_TIMEOUT, MUON_NS_BF16, MUON_NS_FP32, MUON_OK, MuonHyper, MuonNsMatrix,
+                   MuonNsSchedule, MuonParam)
+
+__all__ = ["MuonError", "MuonPlan", "NsPlan", "muon_step", "ns_orthogonalize", "sync_status",
+           "library", "HYBRID_SCHEDULE", "wait_probe", "set_wait_limit_ns"]
+
+# the pages' hybrid schedule: 8 aggressive steps, then 2 standard ones
+HYBRID_SCHEDULE = ((3.4445, -4.7750, 2.0315),) * 8 + ((2.0, -1.5, 0.5),) * 2
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        msg = _lib.load().muon_status_string(status).decode()
+        super().__init__(f"{what}: {msg} (status {status})" if what else msg)
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _check(status: int, what: str):
+    if status != MUON_OK:
+        raise MuonError(status, what)
+
+
+def _precision(p) -> int:
+    if p in ("bf16", MUON_NS_BF16, torch.bfloat16):
+        return MUON_NS_BF16
+    if p in ("fp32", MUON_NS_FP32, torch.float32):
+        return MUON_NS_FP32
+    raise ValueError(f"precision must be 'bf16' or 'fp32', got {p!r}")
+
+
+def _matrix(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.float32 or t.dim() != 2 or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous 2-D float32 tensor")
+    return t
+
+
+def _schedule(schedule, eps):
+    """(struct or None, keep-alive array)."""
+    if schedule is None and eps is None:
+        return None, None
+    sched = HYBRID_SCHEDULE if schedule is None else tuple(tuple(s) for s in schedule)
+    flat = (ctypes.c_float * (3 * len(sched)))(*[float(v) for s in sched for v in s])
+    st = MuonNsSchedule(len(sched), ctypes.cast(flat, ctypes.POINTER(ctypes.c_float)),
+                        1e-7 if eps is None else float(eps))
+    return st, flat
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+class _PlanBase:
+    _plan = None
+
+    def __del__(self):
+        if self._plan:
+            _lib.load().muon_plan_destroy(self._plan)
+            self._plan = None
+
+    @property
+    def workspace_bytes(self) -> int:
+        n = ctypes.c_size_t()
+        _check(_lib.load().muon_plan_workspace_size(self._plan, ctypes.byref(n)), "workspace_size")
+        return n.value
+
+    def alloc_workspace(self, device=None) -> torch.Tensor:
+        device = self.device if device is None else device
+        return torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8, device=device)
+
+    def launches(self):
+        """Kinds of the kernels one execute launches (0 elementwise, 1 Gram,
+        2 polynomial, 3 apply, 4 apply + update)."""
+        lib = _lib.load()
+        n = ctypes.c_int()
+        _check(lib.muon_plan_launches(self._plan, ctypes.byref(n), None, 0), "launches")
+        kinds = (ctypes.c_int * n.value)()
+        _check(lib.muon_plan_launches(self._plan, ctypes.byref(n), kinds, n.value), "launches")
+        return list(kinds)
+
+    def set_events(self, events: Optional[Sequence[torch.cuda.Event]]):
+        """Record events[2k] / events[2k+1] around launch k of every execute."""
+        lib = _lib.load()
+        if not events:
+            _check(lib.muon_plan_set_events(self._plan, None, 0), "set_events")
+            self._events = None
+            return
+        for e in events:
+            e.record()  # materialise the underlying cudaEvent_t
+        handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        _check(lib.muon_plan_set_events(self._plan, handles, len(events)), "set_events")
+        self._events = list(events)
+
+    def flops(self):
+        """Useful FLOPs of one execute per stage kind (Gram, poly, apply)."""
+        g, p, a = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        _check(_lib.load().muon_plan_flops(self._plan, ctypes.byref(g), ctypes.byref(p),
+                                           ctypes.byref(a)), "flops")
+        return g.value, p.value, a.value
+
+    def _ws(self, workspace):
+        if workspace is None:
+            workspace = self._own_ws = getattr(self, "_own_ws", None) or self.alloc_workspace()
+        if workspace.device.type != "cuda":
+            raise TypeError("workspace must be a CUDA tensor")
+        return workspace
+
+
+class MuonPlan(_PlanBase):
+    """A planned Muon step over a fixed list of (W, G, M[, O]) fp32 CUDA matrices."""
+
+    def __init__(self, params: Iterable, precision="bf16", schedule=None, eps=None):
+        items = []
+        self._tensors = []
+        for k, p in enumerate(params):
+            W, G, M = (_matrix(t, f"params[{k}].{nm}") for t, nm in zip(p[:3], "WGM"))
+            O = p[3] if len(p) > 3 else None
+            if O is not None:
+                _matrix(O, f"params[{k}].O")
+            if not (W.shape == G.shape == M.shape and (O is None or O.shape == W.shape)):
+                raise ValueError(f"params[{k}]: W, G, M (and O) must have one shape")
+            n, m = W.shape
+            items.append(MuonParam(W.data_ptr(), G.data_ptr(), M.data_ptr(),
+                                   O.data_ptr() if O is not None else None, n, m))
+            self._tensors.append((W, G, M, O))
+        if not items:
+            raise ValueError("no matrices")
+        self.device = self._tensors[0][0].device
+        arr = (MuonParam * len(items))(*items)
+        sched, self._sched_keep = _schedule(schedule, eps)
+        plan = ctypes.c_void_p()
+        _check(_lib.load().muon_plan_create(arr, len(items), _precision(precision),
+                                            ctypes.byref(sched) if sched else None,
+                                            ctypes.byref(plan)), "muon_plan_create")
+        self._plan = plan
+
+    def execute(self, workspace=None, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2,
+                nesterov=True, stream=None):
+        workspace = self._ws(workspace)
+        h = MuonHyper(lr, momentum, weight_decay, gamma, 1 if nesterov else 0)
+        _check(_lib.load().muon_plan_execute(self._plan, ctypes.byref(h), workspace.data_ptr(),
+                                             workspace.numel(), _stream_ptr(stream)),
+               "muon_plan_execute")
+
+
+class NsPlan(_PlanBase):
+    """A planned ns_orthogonalize over a fixed list of (X, O) fp32 CUDA matrices."""
+
+    def __init__(self, pairs: Iterable, precision="bf16", schedule=None, eps=None):
+        items = []
+        self._tensors = []
+        for k, (X, O) in enumerate(pairs):
+            _matrix(X, f"X[{k}]")
+            _matrix(O, f"O[{k}]")
+            if X.shape != O.shape:
+                raise ValueError(f"X[{k}] and O[{k}] differ in shape")
+            items.append(MuonNsMatrix(X.data_ptr(), O.data_ptr(), X.shape[0], X.shape[1]))
+            self._tensors.append((X, O))
+        if not items:
+            raise ValueError("no matrices")
+        self.device = self._tensors[0][0].device
+        arr = (MuonNsMatrix * len(items))(*items)
+        sched, self._sched_keep = _schedule(schedule, eps)
+        plan = ctypes.c_void_p()
+        _check(_lib.load().muon_plan_create_ns(arr, len(items), _precision(precision),
+                                               ctypes.byref(sched) if sched else None,
+                                               ctypes.byref(plan)), "muon_plan_create_ns")
+        self._plan = plan
+
+    def execute(self, workspace=None, stream=None):
+        workspace = self._ws(workspace)
+        _check(_lib.load().muon_plan_execute(self._plan, None, workspace.data_ptr(),
+                                             workspace.numel(), _stream_ptr(stream)),
+               "muon_plan_execute")
+
+
+def muon_step(params, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True,
+              precision="bf16", schedule=None, eps=None, workspace=None, stream=None):
+    """One-shot Muon step (C ABI muon_step) over a list of (W, G, M[, O])."""
+    items = []
+    keep = []
+    for k, p in enumerate(params):
+        W, G, M = (_matrix(t, f"params[{k}].{nm}") for t, nm in zip(p[:3], "WGM"))
+        O = p[3] if len(p) > 3 else None
+        if not (W.shape == G.shape == M.shape):
+            raise ValueError(f"params[{k}]: W, G, M must have one shape")
+        keep.append(p)
+        items.append(MuonParam(W.data_ptr(), G.data_ptr(), M.data_ptr(),
+                               O.data_ptr() if O is not None else None, *W.shape))
+    arr = (MuonParam * len(items))(*items)
+    lib = _lib.load()
+    prec = _precision(precision)
+    if workspace is None:
+        n = ctypes.c_size_t()
+        _check(lib.muon_workspace_size(arr, len(items), prec, ctypes.byref(n)), "muon_workspace_size")
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=keep[0][0].device)
+    sched, _keep = _schedule(schedule, eps)
+    _check(lib.muon_step(arr, len(items), lr, momentum, weight_decay, gamma, 1 if nesterov else 0,
+                         ctypes.byref(sched) if sched else None, prec, workspace.data_ptr(),
+                         workspace.numel(), _stream_ptr(stream)), "muon_step")
+    return workspace
+
+
+def ns_orthogonalize(xs, out=None, precision="bf16", schedule=None, eps=None, workspace=None,
+                     stream=None):
+    """O' = NewtonSchulz(X / (||X||_F + eps)) per matrix (C ABI ns_orthogonalize)."""
+    xs = [_matrix(x, f"X[{k}]") for k, x in enumerate(xs)]
+    out = [torch.empty_like(x) for x in xs] if out is None else list(out)
+    items = (MuonNsMatrix * len(xs))(*[MuonNsMatrix(x.data_ptr(), o.data_ptr(), *x.shape)
+                                       for x, o in zip(xs, out)])
+    lib = _lib.load()
+    prec = _precision(precision)
+    if workspace is None:
+        n = ctypes.c_size_t()
+        _check(lib.ns_workspace_size(items, len(xs), prec, ctypes.byref(n)), "ns_workspace_size")
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=xs[0].device)
+    sched, _keep = _schedule(schedule, eps)
+    _check(lib.ns_orthogonalize(items, len(xs), ctypes.byref(sched) if sched else None, prec,
+                                workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
+           "ns_orthogonalize")
+    return out
+
+
+def sync_status(stream=None) -> int:
+    """Synchronise and return the device error status (MUON_OK or MUON_ERR_TIMEOUT)."""
+    return _lib.load().muon_sync_status(_stream_ptr(stream))
+
+
+def set_wait_limit_ns(ns: int):
+    _lib.load().muon_set_wait_limit_ns(int(ns))
+
+
+def wait_probe(flag: torch.Tensor, limit_ns: int, stream=None):
+    """Launch one bounded device wait on ``flag`` (int32 CUDA tensor)."""
+    if flag.dtype != torch.int32 or flag.device.type != "cuda":
+        raise TypeError("flag must be an int32 CUDA tensor")
+    _check(_lib.load().muon_wait_probe(flag.data_ptr(), int(limit_ns), _stream_ptr(stream)),
+           "muon_wait_probe")

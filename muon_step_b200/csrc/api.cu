@@ -1,0 +1,615 @@
+// Host planner and C ABI (include/muon_step.h).
+//
+// Planning groups matrices by Newton-Schulz shape (r, c) = (min, max), lays
+// the per-group working buffers out in the caller's workspace, enumerates the
+// tiles of every stage, and keeps a host image of the descriptor tables. An
+// execute copies that image into the workspace the first time it sees the
+// workspace pointer (TMA tensor maps are encoded then, since they embed the
+// buffers' addresses), and then launches 1 + 3 * steps kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <new>
+#include <utility>
+#include <vector>
+
+#include "kernels.cuh"
+#include "muon_step.h"
+#include "ptx_sm100.cuh"
+
+using namespace muon;
+
+namespace {
+
+__device__ int g_device_error;  // per device: error bits of the library's kernels
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+int* g_err_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+int g_cc_major[kMaxDevices] = {};
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+// Per-device setup: the error word's device address and the SM count.
+muon_status_t device_setup(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_err_ptr[dev]) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    g_cc_major[dev] = major;
+    g_num_sms[dev] = sms;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return MUON_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  if (g_cc_major[dev] != 10) return MUON_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  return MUON_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map over a group's [count][rows][ld] buffer, box {64, box_rows, 1},
+// 128-byte swizzle, zero fill outside [inner, rows, count].
+bool encode_bf16_3d(CUtensorMap* out, void* base, int64_t inner, int64_t rows, int64_t ld,
+                    int64_t count, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(count)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2), static_cast<cuuint64_t>(rows * ld * 2)};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+const float kHybrid[10][3] = {{3.4445f, -4.7750f, 2.0315f}, {3.4445f, -4.7750f, 2.0315f},
+                              {3.4445f, -4.7750f, 2.0315f}, {3.4445f, -4.7750f, 2.0315f},
+                              {3.4445f, -4.7750f, 2.0315f}, {3.4445f, -4.7750f, 2.0315f},
+                              {3.4445f, -4.7750f, 2.0315f}, {3.4445f, -4.7750f, 2.0315f},
+                              {2.0f, -1.5f, 0.5f},          {2.0f, -1.5f, 0.5f}};
+
+}  // namespace
+
+struct muon_plan_s {
+  int mode = 0;  // 0: Muon step, 1: ns_orthogonalize
+  muon_precision_t prec = MUON_NS_BF16;
+  int steps = 10;
+  std::vector<float> abc;
+  float eps = 1e-7f;
+  std::vector<GroupDesc> groups;
+  std::vector<MatDesc> mats;  // internal (group-major) order
+  int64_t ew_tiles = 0;
+  int64_t stage_tiles[kNumKinds] = {0, 0, 0};
+  double flops[kNumKinds] = {0, 0, 0};
+  size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_partial = 0, off_counter = 0,
+         off_scale = 0, desc_bytes = 0, ws_bytes = 0;
+  std::vector<uint8_t> blob;
+  void* uploaded_ws = nullptr;
+  int uploaded_dev = -1;
+  std::vector<void*> events;
+};
+
+namespace {
+
+muon_status_t set_schedule(muon_plan_s* p, const muon_ns_schedule_t* s) {
+  if (!s) {
+    p->steps = 10;
+    p->abc.assign(&kHybrid[0][0], &kHybrid[0][0] + 30);
+    p->eps = 1e-7f;
+    return MUON_OK;
+  }
+  if (s->steps < 1 || s->steps > MUON_MAX_NS_STEPS || !s->abc || !(s->eps > 0.f) ||
+      !std::isfinite(s->eps))
+    return MUON_ERR_INVALID_ARG;
+  for (int k = 0; k < 3 * s->steps; ++k)
+    if (!std::isfinite(s->abc[k])) return MUON_ERR_INVALID_ARG;
+  p->steps = s->steps;
+  p->abc.assign(s->abc, s->abc + 3 * s->steps);
+  p->eps = s->eps;
+  return MUON_OK;
+}
+
+// Build groups, tiles, flop counts and the workspace layout from `mats`
+// (caller order; only pointers, n, m filled).
+muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
+  const bool tc = (p->prec == MUON_NS_BF16);
+  std::map<std::pair<int64_t, int64_t>, int> gid;
+  std::vector<std::vector<int>> members;
+  for (size_t k = 0; k < caller.size(); ++k) {
+    const int64_t r = std::min(caller[k].n, caller[k].m), c = std::max(caller[k].n, caller[k].m);
+    auto key = std::make_pair(r, c);
+    auto it = gid.find(key);
+    if (it == gid.end()) {
+      if (static_cast<int>(members.size()) >= kMaxGroups) return MUON_ERR_UNSUPPORTED;
+      it = gid.emplace(key, static_cast<int>(members.size())).first;
+      members.emplace_back();
+    }
+    members[it->second].push_back(static_cast<int>(k));
+  }
+  std::vector<std::pair<int64_t, int64_t>> shape(members.size());
+  for (auto& kv : gid) shape[kv.second] = kv.first;
+
+  p->groups.assign(members.size(), GroupDesc{});
+  p->mats.clear();
+  int64_t ew_total = 0;
+  for (size_t g = 0; g < members.size(); ++g) {
+    GroupDesc& gd = p->groups[g];
+    const int64_t r = shape[g].first, c = shape[g].second;
+    gd.r = static_cast<int32_t>(r);
+    gd.c = static_cast<int32_t>(c);
+    gd.ldc = static_cast<int32_t>(align_up(static_cast<size_t>(c), 8));
+    gd.ldr = static_cast<int32_t>(align_up(static_cast<size_t>(r), 8));
+    gd.count = static_cast<int32_t>(members[g].size());
+    gd.first_mat = static_cast<int32_t>(p->mats.size());
+    double fl[kNumKinds] = {0, 0, 0};
+    if (tc) {
+      const int64_t rb = cdiv(r, kBM);
+      int64_t syrk = 0;
+      for (int64_t i = 0; i < rb; ++i) {
+        syrk += i / 2 + 1;
+        const double rows = static_cast<double>(std::min<int64_t>(kBM, r - i * kBM));
+        for (int64_t bj = 0; bj <= i; ++bj) {  // computed and stored 128 x 128 blocks
+          const double cols = static_cast<double>(std::min<int64_t>(kBM, r - bj * kBM));
+          fl[kGram] += 2.0 * rows * cols * static_cast<double>(c);
+          fl[kPoly] += 2.0 * rows * cols * static_cast<double>(r);
+        }
+      }
+      gd.tiles_per_mat[kGram] = syrk;
+      gd.tiles_per_mat[kPoly] = syrk;
+      gd.tiles_per_mat[kApply] = rb * cdiv(c, kBN);
+    } else {
+      gd.tiles_per_mat[kGram] = cdiv(r, kSBM) * cdiv(r, kSBN);
+      gd.tiles_per_mat[kPoly] = gd.tiles_per_mat[kGram];
+      gd.tiles_per_mat[kApply] = cdiv(r, kSBM) * cdiv(c, kSBN);
+      fl[kGram] = 2.0 * r * r * static_cast<double>(c);
+      fl[kPoly] = 2.0 * r * r * static_cast<double>(r);
+    }
+    fl[kApply] = 2.0 * r * static_cast<double>(c) * static_cast<double>(r);
+    for (int k = 0; k < kNumKinds; ++k) {
+      gd.tile_base[k] = p->stage_tiles[k];
+      p->stage_tiles[k] += gd.tiles_per_mat[k] * gd.count;
+      gd.tile_flops[k] = static_cast<int64_t>(fl[k]);
+      p->flops[k] += fl[k] * gd.count * p->steps;
+    }
+    for (size_t idx = 0; idx < members[g].size(); ++idx) {
+      MatDesc md = caller[members[g][idx]];
+      md.transposed = md.n > md.m ? 1 : 0;
+      md.group = static_cast<int32_t>(g);
+      md.index = static_cast<int32_t>(idx);
+      md.ew_tile_begin = ew_total;
+      md.ew_tiles = cdiv(md.n, kEwRows) * cdiv(md.m, kEwCols);
+      ew_total += md.ew_tiles;
+      p->mats.push_back(md);
+    }
+  }
+  p->ew_tiles = ew_total;
+
+  // workspace layout
+  const size_t ng = p->groups.size(), nm = p->mats.size();
+  size_t off = 0;
+  p->off_groups = off;
+  off = align_up(off + ng * sizeof(GroupDesc), 256);
+  p->off_mats = off;
+  off = align_up(off + nm * sizeof(MatDesc), 256);
+  p->off_tmaps = off;
+  off = align_up(off + (tc ? ng * kTmPerGroup * sizeof(CUtensorMap) : 0), 256);
+  p->off_partial = off;
+  off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
+  p->off_counter = off;
+  off = align_up(off + nm * sizeof(unsigned), 256);
+  p->off_scale = off;
+  off = align_up(off + nm * sizeof(float), 256);
+  p->desc_bytes = off;
+  off = align_up(off, 1024);
+  for (auto& gd : p->groups) {
+    const size_t cnt = static_cast<size_t>(gd.count);
+    const size_t x_elems = cnt * static_cast<size_t>(gd.r) * gd.ldc;
+    const size_t a_elems = cnt * static_cast<size_t>(gd.r) * gd.ldr;
+    const size_t ab_bytes = tc ? 2 : 4;
+    gd.xf_off[0] = static_cast<int64_t>(off);
+    off = align_up(off + x_elems * 4, 1024);
+    if (tc) {
+      gd.xf_off[1] = gd.xf_off[0];
+      gd.xb_off[0] = static_cast<int64_t>(off);
+      off = align_up(off + x_elems * 2, 1024);
+      gd.xb_off[1] = static_cast<int64_t>(off);
+      off = align_up(off + x_elems * 2, 1024);
+    } else {
+      gd.xf_off[1] = static_cast<int64_t>(off);
+      off = align_up(off + x_elems * 4, 1024);
+      gd.xb_off[0] = gd.xb_off[1] = 0;
+    }
+    gd.a_off = static_cast<int64_t>(off);
+    off = align_up(off + a_elems * ab_bytes, 1024);
+    gd.b_off = static_cast<int64_t>(off);
+    off = align_up(off + a_elems * ab_bytes, 1024);
+  }
+  p->ws_bytes = off;
+
+  p->blob.assign(p->desc_bytes, 0);
+  std::memcpy(p->blob.data() + p->off_groups, p->groups.data(), ng * sizeof(GroupDesc));
+  std::memcpy(p->blob.data() + p->off_mats, p->mats.data(), nm * sizeof(MatDesc));
+  return MUON_OK;
+}
+
+bool valid_shape(int64_t n, int64_t m) {
+  return n >= 1 && m >= 1 && n <= 0x7fffffffLL && m <= 0x7fffffffLL;
+}
+
+muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
+  if (p->prec == MUON_NS_BF16) {
+    char* base = static_cast<char*>(ws);
+    auto* maps = reinterpret_cast<CUtensorMap*>(p->blob.data() + p->off_tmaps);
+    for (size_t g = 0; g < p->groups.size(); ++g) {
+      const GroupDesc& gd = p->groups[g];
+      CUtensorMap* m = maps + g * kTmPerGroup;
+      const bool ok =
+          encode_bf16_3d(&m[kTmXb0K], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, kBM) &&
+          encode_bf16_3d(&m[kTmXb1K], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, kBM) &&
+          encode_bf16_3d(&m[kTmXb0MN], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 64) &&
+          encode_bf16_3d(&m[kTmXb1MN], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 64) &&
+          encode_bf16_3d(&m[kTmA], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, kBM) &&
+          encode_bf16_3d(&m[kTmB], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, kBM);
+      if (!ok) return MUON_ERR_CUDA;
+    }
+  }
+  if (cudaMemcpyAsync(ws, p->blob.data(), p->desc_bytes, cudaMemcpyHostToDevice, stream) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  p->uploaded_ws = ws;
+  p->uploaded_dev = dev;
+  return MUON_OK;
+}
+
+muon_status_t record(muon_plan_s* p, int slot, cudaStream_t stream) {
+  if (p->events.empty()) return MUON_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(p->events[slot]), stream) == cudaSuccess
+             ? MUON_OK
+             : MUON_ERR_CUDA;
+}
+
+int launch_count(const muon_plan_s* p) { return 1 + 3 * p->steps; }
+
+}  // namespace
+
+extern "C" {
+
+muon_status_t muon_plan_create(const muon_param_t* params, int count, muon_precision_t prec,
+                               const muon_ns_schedule_t* sched, muon_plan_t* plan) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (!params || count <= 0) return MUON_ERR_INVALID_ARG;
+  if (prec != MUON_NS_BF16 && prec != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
+  std::vector<MatDesc> caller(static_cast<size_t>(count));
+  for (int k = 0; k < count; ++k) {
+    const muon_param_t& q = params[k];
+    if (!q.W || !q.G || !q.M || !valid_shape(q.n, q.m)) return MUON_ERR_INVALID_ARG;
+    MatDesc md{};
+    md.W = q.W;
+    md.G = q.G;
+    md.M = q.M;
+    md.O = q.O;
+    md.n = q.n;
+    md.m = q.m;
+    caller[k] = md;
+  }
+  auto* p = new (std::nothrow) muon_plan_s();
+  if (!p) return MUON_ERR_INVALID_ARG;
+  p->mode = 0;
+  p->prec = prec;
+  muon_status_t st = set_schedule(p, sched);
+  if (st == MUON_OK) st = build_plan(p, caller);
+  if (st != MUON_OK) {
+    delete p;
+    return st;
+  }
+  *plan = p;
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_create_ns(const muon_ns_matrix_t* mats, int count,
+                                  muon_precision_t prec, const muon_ns_schedule_t* sched,
+                                  muon_plan_t* plan) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (!mats || count <= 0) return MUON_ERR_INVALID_ARG;
+  if (prec != MUON_NS_BF16 && prec != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
+  std::vector<MatDesc> caller(static_cast<size_t>(count));
+  for (int k = 0; k < count; ++k) {
+    const muon_ns_matrix_t& q = mats[k];
+    if (!q.X || !q.O || !valid_shape(q.n, q.m)) return MUON_ERR_INVALID_ARG;
+    MatDesc md{};
+    md.G = q.X;
+    md.O = q.O;
+    md.n = q.n;
+    md.m = q.m;
+    caller[k] = md;
+  }
+  auto* p = new (std::nothrow) muon_plan_s();
+  if (!p) return MUON_ERR_INVALID_ARG;
+  p->mode = 1;
+  p->prec = prec;
+  muon_status_t st = set_schedule(p, sched);
+  if (st == MUON_OK) st = build_plan(p, caller);
+  if (st != MUON_OK) {
+    delete p;
+    return st;
+  }
+  *plan = p;
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes) {
+  if (!plan || !bytes) return MUON_ERR_INVALID_ARG;
+  *bytes = plan->ws_bytes;
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds) {
+  if (!plan || !count) return MUON_ERR_INVALID_ARG;
+  const int n = launch_count(plan);
+  *count = n;
+  if (kinds) {
+    for (int k = 0; k < n && k < max_kinds; ++k) {
+      if (k == 0) kinds[k] = 0;
+      else {
+        const int kind = (k - 1) % 3;
+        const bool last = (k - 1) / 3 == plan->steps - 1;
+        kinds[k] = (kind == kApply) ? (last ? 4 : 3) : kind + 1;
+      }
+    }
+  }
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_events(muon_plan_t plan, void* const* events, int count) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  if (count == 0) {
+    plan->events.clear();
+    return MUON_OK;
+  }
+  if (!events || count != 2 * launch_count(plan)) return MUON_ERR_INVALID_ARG;
+  for (int k = 0; k < count; ++k)
+    if (!events[k]) return MUON_ERR_INVALID_ARG;
+  plan->events.assign(events, events + count);
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_flops(muon_plan_t plan, double* gram, double* poly, double* apply) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  if (gram) *gram = plan->flops[kGram];
+  if (poly) *poly = plan->flops[kPoly];
+  if (apply) *apply = plan->flops[kApply];
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, void* workspace,
+                                size_t workspace_bytes, void* stream_ptr) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  if (plan->mode == 0) {
+    if (!hyper) return MUON_ERR_INVALID_ARG;
+    if (!std::isfinite(hyper->lr) || !std::isfinite(hyper->momentum) ||
+        !std::isfinite(hyper->weight_decay) || !std::isfinite(hyper->gamma))
+      return MUON_ERR_INVALID_ARG;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
+      workspace_bytes < plan->ws_bytes)
+    return MUON_ERR_WORKSPACE;
+  int dev = 0;
+  muon_status_t st = device_setup(&dev);
+  if (st != MUON_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (workspace != plan->uploaded_ws || dev != plan->uploaded_dev) {
+    st = upload(plan, workspace, dev, stream);
+    if (st != MUON_OK) return st;
+  }
+  char* ws = static_cast<char*>(workspace);
+  const auto* groups = reinterpret_cast<const GroupDesc*>(ws + plan->off_groups);
+  const auto* mats = reinterpret_cast<const MatDesc*>(ws + plan->off_mats);
+  float* scale = reinterpret_cast<float*>(ws + plan->off_scale);
+  int* err = g_err_ptr[dev];
+  const uint64_t limit = g_wait_limit_ns;
+
+  EwArgs ew{};
+  ew.groups = groups;
+  ew.mats = mats;
+  ew.ws = ws;
+  ew.partial = reinterpret_cast<float*>(ws + plan->off_partial);
+  ew.counter = reinterpret_cast<unsigned*>(ws + plan->off_counter);
+  ew.scale = scale;
+  ew.err = err;
+  ew.total_tiles = plan->ew_tiles;
+  ew.nmats = static_cast<int32_t>(plan->mats.size());
+  ew.mode = plan->mode;
+  ew.nesterov = (plan->mode == 0 && hyper->nesterov) ? 1 : 0;
+  ew.write_bf16 = plan->prec == MUON_NS_BF16 ? 1 : 0;
+  ew.mu = plan->mode == 0 ? hyper->momentum : 0.f;
+  ew.eps = plan->eps;
+  if ((st = record(plan, 0, stream)) != MUON_OK) return st;
+  if (launch_elementwise(ew, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  if ((st = record(plan, 1, stream)) != MUON_OK) return st;
+
+  const bool tc = plan->prec == MUON_NS_BF16;
+  const int sms = g_num_sms[dev];
+  int slot = 2;
+  for (int k = 0; k < plan->steps; ++k) {
+    for (int kind = 0; kind < kNumKinds; ++kind) {
+      StageArgs sa{};
+      sa.groups = groups;
+      sa.mats = mats;
+      sa.tmaps = ws + plan->off_tmaps;
+      sa.ws = ws;
+      sa.scale = scale;
+      sa.err = err;
+      sa.total_tiles = plan->stage_tiles[kind];
+      sa.ngroups = static_cast<int32_t>(plan->groups.size());
+      sa.first = k == 0;
+      sa.last = k == plan->steps - 1;
+      sa.xsrc = k & 1;
+      sa.a = plan->abc[3 * k];
+      sa.b = plan->abc[3 * k + 1];
+      sa.c = plan->abc[3 * k + 2];
+      if (plan->mode == 0) {
+        sa.lr = hyper->lr;
+        sa.wd = hyper->weight_decay;
+        sa.gamma = hyper->gamma;
+      }
+      sa.wait_limit_ns = limit;
+      const int64_t tiles = sa.total_tiles;
+      cudaError_t e;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      if (tc) {
+        const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+        e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, stream);
+      } else {
+        const int grid = static_cast<int>(std::min<int64_t>(tiles, 8LL * sms));
+        e = launch_stage_simt(static_cast<StageKind>(kind), sa, grid, stream);
+      }
+      if (e != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
+  }
+  return MUON_OK;
+}
+
+void muon_plan_destroy(muon_plan_t plan) { delete plan; }
+
+muon_status_t muon_workspace_size(const muon_param_t* params, int count, muon_precision_t prec,
+                                  size_t* bytes) {
+  if (!bytes) return MUON_ERR_INVALID_ARG;
+  muon_plan_t p = nullptr;
+  muon_status_t st = muon_plan_create(params, count, prec, nullptr, &p);
+  if (st != MUON_OK) return st;
+  *bytes = p->ws_bytes;
+  muon_plan_destroy(p);
+  return MUON_OK;
+}
+
+muon_status_t muon_step(const muon_param_t* params, int count, float lr, float momentum,
+                        float weight_decay, float gamma, int nesterov,
+                        const muon_ns_schedule_t* sched, muon_precision_t prec, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  muon_plan_t p = nullptr;
+  muon_status_t st = muon_plan_create(params, count, prec, sched, &p);
+  if (st != MUON_OK) return st;
+  muon_hyper_t h{lr, momentum, weight_decay, gamma, nesterov};
+  st = muon_plan_execute(p, &h, workspace, workspace_bytes, stream);
+  muon_plan_destroy(p);
+  return st;
+}
+
+muon_status_t ns_workspace_size(const muon_ns_matrix_t* mats, int count, muon_precision_t prec,
+                                size_t* bytes) {
+  if (!bytes) return MUON_ERR_INVALID_ARG;
+  muon_plan_t p = nullptr;
+  muon_status_t st = muon_plan_create_ns(mats, count, prec, nullptr, &p);
+  if (st != MUON_OK) return st;
+  *bytes = p->ws_bytes;
+  muon_plan_destroy(p);
+  return MUON_OK;
+}
+
+muon_status_t ns_orthogonalize(const muon_ns_matrix_t* mats, int count,
+                               const muon_ns_schedule_t* sched, muon_precision_t prec,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  muon_plan_t p = nullptr;
+  muon_status_t st = muon_plan_create_ns(mats, count, prec, sched, &p);
+  if (st != MUON_OK) return st;
+  st = muon_plan_execute(p, nullptr, workspace, workspace_bytes, stream);
+  muon_plan_destroy(p);
+  return st;
+}
+
+muon_status_t muon_sync_status(void* stream) {
+  int dev = 0;
+  muon_status_t st = device_setup(&dev);
+  if (st != MUON_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
+  int bits = 0;
+  if (cudaMemcpy(&bits, g_err_ptr[dev], sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (bits) {
+    const int zero = 0;
+    if (cudaMemcpy(g_err_ptr[dev], &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  return (bits & kErrTimeout) ? MUON_ERR_TIMEOUT : MUON_OK;
+}
+
+const char* muon_status_string(muon_status_t status) {
+  switch (status) {
+    case MUON_OK: return "ok";
+    case MUON_ERR_INVALID_ARG: return "invalid argument";
+    case MUON_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MUON_ERR_CUDA: return "CUDA runtime error";
+    case MUON_ERR_UNSUPPORTED: return "unsupported device or size";
+    case MUON_ERR_TIMEOUT: return "device-side wait expired";
+  }
+  return "unknown status";
+}
+
+int muon_abi_version(void) { return MUON_ABI_VERSION; }
+
+void muon_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns < 1000 ? 1000 : ns; }
+
+muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream) {
+  if (!flag) return MUON_ERR_INVALID_ARG;
+  int dev = 0;
+  muon_status_t st = device_setup(&dev);
+  if (st != MUON_OK) return st;
+  return launch_wait_probe(flag, g_err_ptr[dev], limit_ns, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MUON_OK
+             : MUON_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace muon {
+
+namespace {
+__global__ void wait_probe_kernel(const int* flag, int* err, unsigned long long limit_ns) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint64_t it = 0; it < ptx::kSpinBackstop; ++it) {
+    if (*reinterpret_cast<const volatile int*>(flag) != 0) return;
+    if (ptx::globaltimer_ns() - t0 > limit_ns) break;
+    __nanosleep(256);
+  }
+  atomicOr(err, kErrTimeout);
+}
+}  // namespace
+
+cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limit_ns,
+                              cudaStream_t stream) {
+  wait_probe_kernel<<<1, 1, 0, stream>>>(flag, err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

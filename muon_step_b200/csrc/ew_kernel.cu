@@ -1,0 +1,211 @@
+// Elementwise front of the Muon step, one pass over G and M:
+//
+//   M_t = mu M_{t-1} + G_t                  (momentum accumulation)
+//   N_t = mu M_t + G_t                      (Nesterov look-ahead)
+//   X_0 = N_t (or N_t^T when n > m)         (orientation rows <= cols)
+//   s   = 1 / (||N_t||_F + eps)             (Frobenius normalisation scale)
+//
+// "Muon 优化器完全拆解…" (pinghaoyang.com.cn), section "V4 的完整更新公式，逐行拆解",
+// Algorithm 1 steps one and two; "Ch 06 · Muon" §5 Algorithm 1 (momentum,
+// Nesterov and the division by ||N_t||_F). The scale s is not applied here:
+// the first Newton-Schulz step folds s^2 into the Gram matrix and s into the
+// iterate, so the unscaled N is written once, in fp32 and as the bf16 operand.
+//
+// HBM-bound: each element reads G and M (8 B) and writes M, the fp32 iterate
+// and the bf16 operand (10 B). Tiles are 32 x 128 elements; a tile's threads
+// read and write whole 128-byte lines. When the iterate is the transpose, the
+// tile is staged in shared memory so that the transposed writes stay
+// coalesced. Per-tile partial sums of squares go to a buffer; the last tile of
+// each matrix to finish (arrival counter) adds them in a fixed order, in
+// double, so the norm is deterministic.
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+
+namespace muon {
+
+namespace {
+
+__device__ __forceinline__ int find_matrix(const MatDesc* mats, int nmats, int64_t tile) {
+  int lo = 0, hi = nmats - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(&mats[mid].ew_tile_begin) <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+struct alignas(8) Bf16x4 {
+  __nv_bfloat162 lo, hi;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs a) {
+  __shared__ float stage[kEwRows][kEwCols + 1];
+  __shared__ float warp_part[8];
+  __shared__ double warp_part_d[8];
+  __shared__ int is_last;
+
+  const int tid = threadIdx.x;
+  const int64_t tile = blockIdx.x;
+  const int mi = find_matrix(a.mats, a.nmats, tile);
+  const MatDesc md = a.mats[mi];
+  const GroupDesc& gd = a.groups[md.group];
+  const int64_t n = md.n, m = md.m;
+  const int64_t col_tiles = (m + kEwCols - 1) / kEwCols;
+  const int64_t local = tile - md.ew_tile_begin;
+  const int64_t row0 = (local / col_tiles) * kEwRows;
+  const int64_t col0 = (local % col_tiles) * kEwCols;
+
+  const int64_t ldc = gd.ldc;
+  const int64_t mat_elems = static_cast<int64_t>(gd.r) * ldc;
+  float* xf = reinterpret_cast<float*>(a.ws + gd.xf_off[0]) + md.index * mat_elems;
+  __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xb_off[0]) + md.index * mat_elems;
+  const bool transposed = md.transposed != 0;
+  const float mu = a.mu;
+  float sumsq = 0.f;
+
+  // N for one element: momentum update written back, look-ahead returned.
+  auto step = [&](float g, float mprev, float* mdst) -> float {
+    if (a.mode != 0) return g;
+    const float mt = fmaf(mu, mprev, g);
+    *mdst = mt;
+    return a.nesterov ? fmaf(mu, mt, g) : mt;
+  };
+
+  const bool vec = ((m & 3) == 0) &&
+                   (((reinterpret_cast<uintptr_t>(md.G) | reinterpret_cast<uintptr_t>(md.M)) & 15) == 0);
+  if (vec) {
+    // thread -> 4 consecutive columns, rows (tid / 32) + 8 k
+    const int c4 = (tid & 31) * 4;
+    const int64_t col = col0 + c4;
+#pragma unroll
+    for (int k = 0; k < kEwRows / 8; ++k) {
+      const int rr = (tid >> 5) + 8 * k;
+      const int64_t row = row0 + rr;
+      float nv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (row < n && col < m) {  // m % 4 == 0: the 4 columns are all in range
+        const int64_t off = row * m + col;
+        const float4 g4 = __ldcs(reinterpret_cast<const float4*>(md.G + off));
+        float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (a.mode == 0) m4 = __ldcs(reinterpret_cast<const float4*>(md.M + off));
+        float4 mo;
+        nv[0] = step(g4.x, m4.x, &mo.x);
+        nv[1] = step(g4.y, m4.y, &mo.y);
+        nv[2] = step(g4.z, m4.z, &mo.z);
+        nv[3] = step(g4.w, m4.w, &mo.w);
+        if (a.mode == 0) __stcs(reinterpret_cast<float4*>(md.M + off), mo);
+        sumsq += nv[0] * nv[0] + nv[1] * nv[1] + nv[2] * nv[2] + nv[3] * nv[3];
+        if (!transposed) {
+          const int64_t xo = row * ldc + col;
+          *reinterpret_cast<float4*>(xf + xo) = make_float4(nv[0], nv[1], nv[2], nv[3]);
+          if (a.write_bf16) {
+            Bf16x4 p;
+            p.lo = __floats2bfloat162_rn(nv[0], nv[1]);
+            p.hi = __floats2bfloat162_rn(nv[2], nv[3]);
+            *reinterpret_cast<Bf16x4*>(xb + xo) = p;
+          }
+        }
+      }
+      if (transposed) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) stage[rr][c4 + e] = nv[e];
+      }
+    }
+  } else {
+    // scalar path: thread -> one column, rows (tid / 128) + 2 k
+    const int cc = tid & (kEwCols - 1);
+    const int64_t col = col0 + cc;
+    for (int k = 0; k < kEwRows / 2; ++k) {
+      const int rr = (tid >> 7) + 2 * k;
+      const int64_t row = row0 + rr;
+      float nv = 0.f;
+      if (row < n && col < m) {
+        const int64_t off = row * m + col;
+        const float g = __ldcs(md.G + off);
+        const float mp = (a.mode == 0) ? __ldcs(md.M + off) : 0.f;
+        float mo;
+        nv = step(g, mp, &mo);
+        if (a.mode == 0) __stcs(md.M + off, mo);
+        sumsq += nv * nv;
+        if (!transposed) {
+          const int64_t xo = row * ldc + col;
+          xf[xo] = nv;
+          if (a.write_bf16) xb[xo] = __float2bfloat16_rn(nv);
+        }
+      }
+      if (transposed) stage[rr][cc] = nv;
+    }
+  }
+
+  if (transposed) {
+    // iterate row j = caller column, iterate column i = caller row
+    __syncthreads();
+    const int w = tid >> 5, lane = tid & 31;
+    const int64_t i = row0 + lane;
+#pragma unroll 4
+    for (int q = 0; q < kEwCols / 8; ++q) {
+      const int cc = w * (kEwCols / 8) + q;
+      const int64_t j = col0 + cc;
+      if (j < m && i < n) {
+        const float v = stage[lane][cc];
+        const int64_t xo = j * ldc + i;
+        xf[xo] = v;
+        if (a.write_bf16) xb[xo] = __float2bfloat16_rn(v);
+      }
+    }
+  }
+
+  // tile partial sum of squares
+  sumsq = warp_sum(sumsq);
+  if ((tid & 31) == 0) warp_part[tid >> 5] = sumsq;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += warp_part[w];
+    a.partial[tile] = s;
+    __threadfence();
+    const unsigned prev = atomicAdd(&a.counter[mi], 1u);
+    is_last = (prev + 1 == static_cast<unsigned>(md.ew_tiles));
+  }
+  __syncthreads();
+  if (!is_last) return;
+
+  // last tile of this matrix: fixed-order double sum of the partials
+  __threadfence();
+  double acc = 0.0;
+  for (int64_t k = tid; k < md.ew_tiles; k += blockDim.x)
+    acc += static_cast<double>(__ldcg(a.partial + md.ew_tile_begin + k));
+  acc = warp_sum_d(acc);
+  if ((tid & 31) == 0) warp_part_d[tid >> 5] = acc;
+  __syncthreads();
+  if (tid == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 8; ++w) s += warp_part_d[w];
+    a.scale[mi] = static_cast<float>(1.0 / (sqrt(s) + static_cast<double>(a.eps)));
+    a.counter[mi] = 0u;
+  }
+}
+
+cudaError_t launch_elementwise(const EwArgs& args, cudaStream_t stream) {
+  if (args.total_tiles <= 0) return cudaSuccess;
+  if (args.total_tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  ew_kernel<<<static_cast<unsigned>(args.total_tiles), 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

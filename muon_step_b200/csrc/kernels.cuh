@@ -1,0 +1,32 @@
+// Launchers of the library's kernels (host side, C++ linkage, internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "muon_internal.h"
+
+namespace muon {
+
+// Momentum + Nesterov (or plain input) + per-tile sums of squares + write of
+// the Newton-Schulz iterate in its orientation; the last tile of each matrix
+// turns the partial sums into the normalisation scale.
+cudaError_t launch_elementwise(const EwArgs& args, cudaStream_t stream);
+
+// One Newton-Schulz stage over every matrix of the plan, bf16 operands on
+// the tcgen05 tensor cores (TMA -> shared memory -> MMA -> TMEM -> epilogue).
+cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid,
+                            cudaStream_t stream);
+
+// The same stage in fp32 on the CUDA cores (validation precision).
+cudaError_t launch_stage_simt(StageKind kind, const StageArgs& args, int grid,
+                              cudaStream_t stream);
+
+// Dynamic shared memory the tcgen05 stage kernels need.
+size_t stage_tc_smem_bytes();
+
+// Bounded wait on a host-visible word that nothing sets: used by the tests of
+// the timeout path. Sets the timeout bit of `err` when the limit passes.
+cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limit_ns,
+                              cudaStream_t stream);
+
+}  // namespace muon

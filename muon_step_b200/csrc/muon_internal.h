@@ -1,0 +1,111 @@
+// Internal descriptor tables shared by the host planner and the device kernels.
+//
+// A Muon step (or an ns_orthogonalize call) over many matrices is planned once
+// on the host: matrices are grouped by their Newton-Schulz shape (r, c) with
+// r = min(n, m) <= c = max(n, m); each group's working buffers sit in one
+// contiguous slab of the caller's workspace so that one 3-D TMA tensor map per
+// buffer covers the whole group. Tile counts per stage kind are prefix-summed
+// over the groups so that a single persistent launch per stage walks every
+// matrix's tiles.
+#pragma once
+
+#include <cstdint>
+
+namespace muon {
+
+constexpr int kMaxGroups = 64;
+constexpr int kMaxSteps = 64;
+
+// tcgen05 tile shape: 128 x 256 output tiles, K blocks of 64 bf16 (128 B).
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+
+// fp32 validation tile shape.
+constexpr int kSBM = 64;
+constexpr int kSBN = 64;
+constexpr int kSBK = 16;
+
+// elementwise (momentum / norm / cast) tile: 32 rows x 128 columns.
+constexpr int kEwRows = 32;
+constexpr int kEwCols = 128;
+
+enum StageKind : int { kGram = 0, kPoly = 1, kApply = 2, kNumKinds = 3 };
+
+// tensor maps per group (bf16 mode)
+enum TmapSlot : int {
+  kTmXb0K = 0,   // X bf16 buffer 0, box {64 cols, 128 rows}: K-major operand
+  kTmXb1K = 1,   // X bf16 buffer 1
+  kTmXb0MN = 2,  // X bf16 buffer 0, box {64 cols, 64 rows}: MN-major operand
+  kTmXb1MN = 3,  // X bf16 buffer 1
+  kTmA = 4,      // Gram matrix A, box {64, 128}
+  kTmB = 5,      // polynomial B = bA + cA^2, box {64, 128}
+  kTmPerGroup = 6
+};
+
+struct GroupDesc {
+  int32_t r, c;          // Newton-Schulz shape, r <= c
+  int32_t ldc, ldr;      // leading dimensions (elements) of r x c and r x r buffers
+  int32_t count;         // matrices in this group
+  int32_t first_mat;     // internal index of the group's first matrix
+  int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate (fp32 mode ping-pongs)
+  int64_t xb_off[2];     // bf16 iterate, ping-pong
+  int64_t a_off, b_off;  // A = X X^T and B = bA + cA^2 (bf16, or fp32 in fp32 mode)
+  int64_t tiles_per_mat[kNumKinds];
+  int64_t tile_base[kNumKinds];
+  int64_t tile_flops[kNumKinds];  // useful FLOPs per matrix per stage (host statistics)
+};
+
+struct MatDesc {
+  float* W;              // caller's weight (n x m, row-major), updated in place
+  const float* G;        // caller's gradient, or the ns_orthogonalize input X
+  float* M;              // caller's momentum buffer (NULL for ns_orthogonalize)
+  float* O;              // optional output O' in the caller's orientation
+  int64_t n, m;          // caller's shape
+  int32_t transposed;    // Newton-Schulz runs on the transpose (n > m)
+  int32_t group;         // shape group
+  int32_t index;         // index within the group
+  int32_t pad0;
+  int64_t ew_tile_begin; // first elementwise tile of this matrix
+  int64_t ew_tiles;      // number of elementwise tiles
+};
+
+// Per-launch arguments of the Newton-Schulz stage kernels.
+struct StageArgs {
+  const GroupDesc* groups;
+  const MatDesc* mats;
+  const void* tmaps;      // CUtensorMap[ngroups][kTmPerGroup], 64-byte aligned
+  char* ws;               // workspace base
+  const float* scale;     // per-matrix 1 / (||N||_F + eps)
+  int* err;               // device error word
+  int64_t total_tiles;
+  int32_t ngroups;
+  int32_t first;          // first Newton-Schulz step: fold the normalisation scale
+  int32_t last;           // last step: write O' and update W instead of the iterate
+  int32_t xsrc;           // which ping-pong buffer holds the current iterate
+  float a, b, c;          // this step's coefficients
+  float lr, wd, gamma;    // update hyper-parameters (last step)
+  uint64_t wait_limit_ns; // bound on every spin-wait
+};
+
+// Elementwise-stage arguments (momentum + Nesterov + Frobenius partials + cast).
+struct EwArgs {
+  const GroupDesc* groups;
+  const MatDesc* mats;
+  char* ws;
+  float* partial;         // one partial sum of squares per elementwise tile
+  unsigned* counter;      // per-matrix arrival counter (left at zero)
+  float* scale;           // per-matrix output 1 / (||N||_F + eps)
+  int* err;
+  int64_t total_tiles;
+  int32_t nmats;
+  int32_t mode;           // 0: Muon (momentum + Nesterov), 1: plain normalisation of G
+  int32_t nesterov;
+  int32_t write_bf16;     // bf16 mode writes the bf16 operand copy too
+  float mu, eps;
+};
+
+// error bits in the device error word
+enum ErrBits : int { kErrTimeout = 1, kErrBadTile = 2 };
+
+}  // namespace muon

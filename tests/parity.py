@@ -1,0 +1,86 @@
+"""Helpers shared by the GPU parity tests: run the library on a workload and
+compare every (or a sampled) matrix with the float64 oracle."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import muon_oracle
+
+# tolerances (relative Frobenius error per matrix)
+TOL_O = {"bf16": 2e-2, "fp32": 1e-4}   # O' against the oracle
+TOL_ELEMENTWISE = 1e-6                  # momentum, and the update given the GPU's own O'
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    if nb == 0.0:
+        return float(np.linalg.norm(a))
+    return float(np.linalg.norm(a - b) / nb)
+
+
+def run_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1):
+    """Snapshot the sampled inputs, run `steps` Muon steps through the library
+    (plan API) capturing O', and return per-sample records."""
+    import muon_step_b200 as ms
+
+    hyper = dict(wl.hyper if hyper is None else hyper)
+    idx = list(range(wl.count)) if sample is None else list(sample)
+    before = {k: (wl.W[k].double().cpu().numpy(), wl.G[k].double().cpu().numpy(),
+                  wl.M[k].double().cpu().numpy()) for k in idx}
+    O = {k: torch.empty_like(wl.W[k]) for k in idx}
+    params = [(wl.W[k], wl.G[k], wl.M[k], O.get(k)) for k in range(wl.count)]
+    plan = ms.MuonPlan(params, precision=precision, schedule=schedule)
+    ws = plan.alloc_workspace()
+    history = []
+    for _ in range(steps):
+        plan.execute(ws, lr=hyper["lr"], momentum=hyper["mu"], weight_decay=hyper["wd"],
+                     gamma=hyper["gamma"], nesterov=hyper["nesterov"])
+        history.append({k: O[k].double().cpu().numpy() for k in idx})
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    after = {k: (wl.W[k].double().cpu().numpy(), wl.M[k].double().cpu().numpy()) for k in idx}
+    return before, after, history, hyper
+
+
+def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1):
+    """Compare the library's step(s) with the oracle; return worst errors."""
+    before, after, history, hyper = run_step(wl, precision, hyper, schedule, sample, steps)
+    sched = muon_oracle.HYBRID_SCHEDULE if schedule is None else schedule
+    worst = {"O": 0.0, "M": 0.0, "W_given_O": 0.0, "W": 0.0}
+    for k, (W, G, M) in before.items():
+        n, m = W.shape
+        for s in range(steps):
+            W, M, O_ref = muon_oracle.muon_step(W, G, M, lr=hyper["lr"], mu=hyper["mu"],
+                                                wd=hyper["wd"], gamma=hyper["gamma"],
+                                                nesterov_on=hyper["nesterov"], schedule=sched)
+            worst["O"] = max(worst["O"], rel(history[s][k], O_ref))
+        W_gpu, M_gpu = after[k]
+        worst["M"] = max(worst["M"], rel(M_gpu, M))
+        worst["W"] = max(worst["W"], rel(W_gpu, W))
+        if steps == 1:
+            # the update arithmetic, given the library's own O'
+            W0 = before[k][0]
+            W_from_O = muon_oracle.decay_and_update(
+                W0, muon_oracle.rescale(history[0][k], n, m, hyper["gamma"]), hyper["lr"], hyper["wd"])
+            worst["W_given_O"] = max(worst["W_given_O"], rel(W_gpu, W_from_O))
+    return worst
+
+
+def check_ns(xs, precision="bf16", schedule=None, eps=1e-7):
+    import muon_step_b200 as ms
+
+    sched = muon_oracle.HYBRID_SCHEDULE if schedule is None else schedule
+    outs = ms.ns_orthogonalize(xs, precision=precision, schedule=schedule, eps=None if eps == 1e-7 else eps)
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    worst = 0.0
+    for x, o in zip(xs, outs):
+        ref = muon_oracle.ns_orthogonalize(x.double().cpu().numpy(), sched, eps)
+        worst = max(worst, rel(o.double().cpu().numpy(), ref))
+    return worst

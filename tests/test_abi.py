@@ -1,0 +1,203 @@
+"""Host-side checks of the C ABI: the library loads and exports every symbol
+the header declares; planning (host only) validates arguments, sizes the
+workspace and counts tiles and FLOPs; no call here touches a GPU."""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from muon_step_b200 import _lib
+from muon_step_b200._lib import (MUON_ERR_INVALID_ARG, MUON_ERR_WORKSPACE, MUON_NS_BF16,
+                                 MUON_NS_FP32, MUON_OK, MuonHyper, MuonNsMatrix, MuonNsSchedule,
+                                 MuonParam)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon_step.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from muon_step_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MUON_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert header_symbols() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_no_other_exported_api_symbols(lib):
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    api = {s for s in exported if s.startswith(("muon_", "ns_"))}
+    assert api == set(header_symbols())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.muon_abi_version() == 1
+    for s in range(6):
+        assert lib.muon_status_string(s)
+    assert lib.muon_status_string(99) == b"unknown status"
+
+
+FAKE = 0x10000  # plan creation records pointers but never dereferences them
+
+
+def params(shapes, with_o=False):
+    arr = (MuonParam * len(shapes))()
+    for k, (n, m) in enumerate(shapes):
+        base = FAKE * (4 * k + 1)
+        arr[k] = MuonParam(base, base + 1 * FAKE, base + 2 * FAKE, base + 3 * FAKE if with_o else None, n, m)
+    return arr
+
+
+def create(lib, shapes, prec=MUON_NS_BF16, sched=None):
+    plan = ctypes.c_void_p()
+    st = lib.muon_plan_create(params(shapes), len(shapes), prec, sched, ctypes.byref(plan))
+    return st, plan
+
+
+def test_plan_rejects_bad_arguments(lib):
+    plan = ctypes.c_void_p()
+    assert lib.muon_plan_create(None, 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_create(params([(4, 4)]), 0, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_create(params([(4, 4)]), 1, 7, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_create(params([(0, 4)]), 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_create(params([(4, -1)]), 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    bad = params([(4, 4)])
+    bad[0].G = None
+    assert lib.muon_plan_create(bad, 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_create(params([(4, 4)]), 1, 0, None, None) == MUON_ERR_INVALID_ARG
+    # schedules: zero steps, too many steps, eps <= 0, NaN coefficient
+    abc = (ctypes.c_float * 6)(1, 0, 0, 1, 0, 0)
+    p = ctypes.cast(abc, ctypes.POINTER(ctypes.c_float))
+    for s in (MuonNsSchedule(0, p, 1e-7), MuonNsSchedule(65, p, 1e-7), MuonNsSchedule(2, p, 0.0),
+              MuonNsSchedule(2, None, 1e-7)):
+        assert create(lib, [(4, 4)], sched=ctypes.byref(s))[0] == MUON_ERR_INVALID_ARG
+    abc[4] = float("nan")
+    assert create(lib, [(4, 4)], sched=ctypes.byref(MuonNsSchedule(2, p, 1e-7)))[0] == MUON_ERR_INVALID_ARG
+
+
+def test_execute_rejects_bad_workspace_without_touching_the_device(lib):
+    st, plan = create(lib, [(64, 96)])
+    assert st == MUON_OK
+    try:
+        n = ctypes.c_size_t()
+        lib.muon_plan_workspace_size(plan, ctypes.byref(n))
+        h = MuonHyper(0.02, 0.95, 0.1, 0.2, 1)
+        assert lib.muon_plan_execute(plan, ctypes.byref(h), None, n.value, None) == MUON_ERR_WORKSPACE
+        assert lib.muon_plan_execute(plan, ctypes.byref(h), FAKE + 128, n.value, None) == MUON_ERR_WORKSPACE
+        assert lib.muon_plan_execute(plan, ctypes.byref(h), FAKE, n.value - 1, None) == MUON_ERR_WORKSPACE
+        assert lib.muon_plan_execute(plan, None, FAKE, n.value, None) == MUON_ERR_INVALID_ARG
+        nan = MuonHyper(float("nan"), 0.95, 0.1, 0.2, 1)
+        assert lib.muon_plan_execute(plan, ctypes.byref(nan), FAKE, n.value, None) == MUON_ERR_INVALID_ARG
+    finally:
+        lib.muon_plan_destroy(plan)
+
+
+def syrk_tiles(r):
+    rb = math.ceil(r / 128)
+    return sum(i // 2 + 1 for i in range(rb))
+
+
+def expected_workspace(shapes, prec):
+    """Independent restatement of the documented layout: per shape group an
+    fp32 iterate (two in fp32 mode), two bf16 iterates (bf16 mode), A and B;
+    rows padded to multiples of 8 elements; regions 1024-byte aligned."""
+    groups = {}
+    for n, m in shapes:
+        groups.setdefault((min(n, m), max(n, m)), []).append((n, m))
+    al = lambda x, a: (x + a - 1) // a * a
+    ng, nm = len(groups), len(shapes)
+    ew = sum(math.ceil(n / 32) * math.ceil(m / 128) for n, m in shapes)
+    off = al(ng * 144, 256)          # GroupDesc is 144 bytes
+    off = al(off + nm * 80, 256)     # MatDesc is 80 bytes
+    off = al(off + (ng * 6 * 128 if prec == MUON_NS_BF16 else 0), 256)
+    off = al(off + ew * 4, 256)
+    off = al(off + nm * 4, 256)
+    off = al(off + nm * 4, 256)
+    off = al(off, 1024)
+    for (r, c), mem in groups.items():
+        k = len(mem)
+        x = k * r * al(c, 8)
+        a = k * r * al(r, 8)
+        if prec == MUON_NS_BF16:
+            for nbytes in (4 * x, 2 * x, 2 * x, 2 * a, 2 * a):
+                off = al(off + nbytes, 1024)
+        else:
+            for nbytes in (4 * x, 4 * x, 4 * a, 4 * a):
+                off = al(off + nbytes, 1024)
+    return off
+
+
+@pytest.mark.parametrize("prec", [MUON_NS_BF16, MUON_NS_FP32])
+def test_workspace_size_matches_layout(lib, prec):
+    shapes = [(256, 512), (512, 256), (7, 3), (1000, 130), (130, 1000), (1, 1)]
+    shapes += [(k, 2 * k + 1) for k in range(2, 40)]  # many groups: descriptor bytes matter
+    st, plan = create(lib, shapes, prec)
+    assert st == MUON_OK
+    n = ctypes.c_size_t()
+    assert lib.muon_plan_workspace_size(plan, ctypes.byref(n)) == MUON_OK
+    lib.muon_plan_destroy(plan)
+    assert n.value == expected_workspace(shapes, prec)
+    m = ctypes.c_size_t()
+    assert lib.muon_workspace_size(params(shapes), len(shapes), prec, ctypes.byref(m)) == MUON_OK
+    assert m.value == n.value
+
+
+def test_launch_list(lib):
+    st, plan = create(lib, [(64, 64)])
+    cnt = ctypes.c_int()
+    kinds = (ctypes.c_int * 64)()
+    assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 64) == MUON_OK
+    lib.muon_plan_destroy(plan)
+    assert cnt.value == 31
+    assert list(kinds[:31]) == [0] + [1, 2, 3] * 9 + [1, 2, 4]
+
+
+def test_flops_count_the_computed_tiles(lib):
+    """Tensor-core mode: Gram and polynomial count the 128 x 128 blocks on and
+    below the diagonal; apply is dense: 2 r^2 c per step."""
+    for r, c in [(256, 512), (1024, 1024), (300, 1000), (4096, 14336)]:
+        st, plan = create(lib, [(r, c)])
+        g, p, a = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        lib.muon_plan_flops(plan, ctypes.byref(g), ctypes.byref(p), ctypes.byref(a))
+        lib.muon_plan_destroy(plan)
+        rb = math.ceil(r / 128)
+        lower = sum(min(128, r - 128 * i) * min(128, r - 128 * j) for i in range(rb) for j in range(i + 1))
+        assert g.value == pytest.approx(10 * 2 * lower * c)
+        assert p.value == pytest.approx(10 * 2 * lower * r)
+        assert a.value == pytest.approx(10 * 2 * r * r * c)
+        # the lower triangle with its diagonal blocks: r^2/2 <= lower <= r^2/2 + 64 r
+        assert r * r / 2 <= lower <= r * r / 2 + 64 * r
+
+
+def test_ns_plan_arguments(lib):
+    plan = ctypes.c_void_p()
+    mats = (MuonNsMatrix * 1)(MuonNsMatrix(FAKE, 2 * FAKE, 5, 9))
+    assert lib.muon_plan_create_ns(mats, 1, MUON_NS_BF16, None, ctypes.byref(plan)) == MUON_OK
+    lib.muon_plan_destroy(plan)
+    mats[0].O = None
+    assert lib.muon_plan_create_ns(mats, 1, MUON_NS_BF16, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+
+
+def test_timing_events_need_two_per_launch(lib):
+    st, plan = create(lib, [(8, 8)])
+    ev = (ctypes.c_void_p * 62)(*([FAKE] * 62))
+    assert lib.muon_plan_set_events(plan, ev, 61) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_set_events(plan, ev, 62) == MUON_OK
+    assert lib.muon_plan_set_events(plan, None, 0) == MUON_OK
+    lib.muon_plan_destroy(plan)

@@ -1,0 +1,118 @@
+"""Parity of the CUDA path with the float64 oracle on seeded inputs.
+
+Tolerances (relative Frobenius error per matrix): O' <= 2e-2 with bf16
+tensor-core operands, <= 1e-4 in the fp32 validation precision; the momentum
+buffer and the update (given the library's own O') <= 1e-6.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests.parity import TOL_ELEMENTWISE, TOL_O, check_ns, check_step, rel
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = [(1, 1), (1, 7), (7, 1), (3, 5), (5, 3), (64, 64), (129, 257), (257, 129),
+          (130, 130), (300, 1000), (1000, 300), (7, 1500), (128, 256), (384, 640)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available()
+    import muon_step_b200 as ms
+    ms.library()
+    yield
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_single_256x512(precision):
+    wl = workloads.make("single_256x512", device="cuda")
+    worst = check_step(wl, precision)
+    assert worst["O"] <= TOL_O[precision], worst
+    assert worst["M"] <= TOL_ELEMENTWISE, worst
+    assert worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("spectrum", ["geometric", "flat"])
+def test_ragged_mixed_shapes(precision, spectrum):
+    wl = workloads.make_random(RAGGED, device="cuda", seed=7, spectrum=spectrum)
+    worst = check_step(wl, precision)
+    assert worst["O"] <= TOL_O[precision], worst
+    assert worst["M"] <= TOL_ELEMENTWISE, worst
+    assert worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_ns_orthogonalize(precision):
+    g = torch.Generator(device="cuda").manual_seed(3)
+    xs = [torch.randn(n, m, device="cuda", generator=g) for n, m in RAGGED]
+    assert check_ns(xs, precision) <= TOL_O[precision]
+
+
+def test_zero_matrix_is_pure_decay():
+    n, m = 200, 333
+    W = torch.randn(n, m, device="cuda")
+    W0 = W.double().cpu().numpy()
+    G = torch.zeros(n, m, device="cuda")
+    M = torch.zeros(n, m, device="cuda")
+    O = torch.full((n, m), 7.0, device="cuda")
+    import muon_step_b200 as ms
+    ms.muon_step([(W, G, M, O)], lr=0.02, weight_decay=0.1)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(O).item() == 0
+    assert torch.count_nonzero(M).item() == 0
+    assert rel(W.double().cpu().numpy(), W0 * (1 - 0.02 * 0.1)) <= TOL_ELEMENTWISE
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_nesterov_off_and_other_hyper(precision):
+    wl = workloads.make_random([(96, 160), (160, 96)], device="cuda", seed=9)
+    hyper = dict(lr=0.05, mu=0.9, wd=0.01, gamma=0.18, nesterov=False)
+    worst = check_step(wl, precision, hyper=hyper)
+    assert worst["O"] <= TOL_O[precision], worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_five_step_quintic_schedule(precision):
+    sched = ((3.4445, -4.7750, 2.0315),) * 5
+    wl = workloads.make_random([(200, 520), (520, 200)], device="cuda", seed=11)
+    worst = check_step(wl, precision, schedule=sched)
+    assert worst["O"] <= TOL_O[precision], worst
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_three_consecutive_steps(precision):
+    wl = workloads.make_random([(256, 384), (384, 256)], device="cuda", seed=13)
+    worst = check_step(wl, precision, steps=3)
+    assert worst["O"] <= TOL_O[precision], worst
+    assert worst["M"] <= TOL_ELEMENTWISE, worst
+
+
+def test_batch64_1024_sampled():
+    """The benchmark's workload at full size (64 x 1024 x 1024, one grouped
+    launch per stage); 6 matrices checked against the oracle."""
+    wl = workloads.make("batch64_1024", device="cuda")
+    sample = [0, 1, 17, 31, 48, 63]
+    worst = check_step(wl, "bf16", sample=sample)
+    assert worst["O"] <= TOL_O["bf16"], worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+def test_timeout_is_reported_and_the_context_survives():
+    import muon_step_b200 as ms
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ms.wait_probe(flag, 2_000_000)  # 2 ms, nothing sets the flag
+    assert ms.sync_status() == 5    # MUON_ERR_TIMEOUT
+    assert ms.sync_status() == 0    # cleared
+    flag.fill_(1)
+    ms.wait_probe(flag, 2_000_000)
+    assert ms.sync_status() == 0
+    # the device still runs the library's kernels
+    wl = workloads.make_random([(64, 96)], device="cuda", seed=1)
+    assert check_step(wl, "bf16")["O"] <= TOL_O["bf16"]
