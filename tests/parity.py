@@ -14,6 +14,20 @@ from oracle import muon_oracle
 TOL_O = {"bf16": 2e-2, "fp32": 1e-4}   # O' against the oracle
 TOL_ELEMENTWISE = 1e-6                  # momentum, and the update given the GPU's own O'
 
+# Matrices with fewer elements than this are too small for the bf16 rounding
+# of the iterate operand to average out over the Frobenius norm: a CPU
+# emulation of the kernels' rounding (bf16 X, A, B; fp32 master iterate) on
+# 12,000 random Gaussian matrices of 2 to 64 elements reached 3.8e-2.
+TINY_ELEMENTS = 256
+TOL_O_TINY_BF16 = 5e-2
+
+
+def tol_o(precision, shape):
+    n, m = shape
+    if precision == "bf16" and n * m < TINY_ELEMENTS:
+        return TOL_O_TINY_BF16
+    return TOL_O[precision]
+
 
 def rel(a, b):
     a = np.asarray(a, dtype=np.float64)
@@ -52,14 +66,16 @@ def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, ste
     """Compare the library's step(s) with the oracle; return worst errors."""
     before, after, history, hyper = run_step(wl, precision, hyper, schedule, sample, steps)
     sched = muon_oracle.HYBRID_SCHEDULE if schedule is None else schedule
-    worst = {"O": 0.0, "M": 0.0, "W_given_O": 0.0, "W": 0.0}
+    worst = {"O": 0.0, "O_over_tol": 0.0, "M": 0.0, "W_given_O": 0.0, "W": 0.0}
     for k, (W, G, M) in before.items():
         n, m = W.shape
         for s in range(steps):
             W, M, O_ref = muon_oracle.muon_step(W, G, M, lr=hyper["lr"], mu=hyper["mu"],
                                                 wd=hyper["wd"], gamma=hyper["gamma"],
                                                 nesterov_on=hyper["nesterov"], schedule=sched)
-            worst["O"] = max(worst["O"], rel(history[s][k], O_ref))
+            e = rel(history[s][k], O_ref)
+            worst["O"] = max(worst["O"], e)
+            worst["O_over_tol"] = max(worst["O_over_tol"], e / tol_o(precision, (n, m)))
         W_gpu, M_gpu = after[k]
         worst["M"] = max(worst["M"], rel(M_gpu, M))
         worst["W"] = max(worst["W"], rel(W_gpu, W))
@@ -79,8 +95,12 @@ def check_ns(xs, precision="bf16", schedule=None, eps=1e-7):
     outs = ms.ns_orthogonalize(xs, precision=precision, schedule=schedule, eps=None if eps == 1e-7 else eps)
     torch.cuda.synchronize()
     assert ms.sync_status() == 0
-    worst = 0.0
+    errs = []
     for x, o in zip(xs, outs):
         ref = muon_oracle.ns_orthogonalize(x.double().cpu().numpy(), sched, eps)
-        worst = max(worst, rel(o.double().cpu().numpy(), ref))
-    return worst
+        errs.append((tuple(x.shape), rel(o.double().cpu().numpy(), ref), tol_o(precision, tuple(x.shape))))
+    return errs
+
+
+def all_within(errs):
+    return all(e <= t for _, e, t in errs)
