@@ -193,6 +193,35 @@ MUON_API void muon_set_wait_limit_ns(uint64_t ns);
  * bit, which muon_sync_status() then reports. */
 MUON_API muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream);
 
+/* ---------------------------------------------------------------- no allocation
+ * The pages describe no counterpart of this entry point; it serves callers
+ * that cannot allocate device memory during a step: runtimes that reserve
+ * (nearly) all of HBM up front for their own pool, real-time or multi-stream
+ * code that cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree may cause, plugins handed data pointers but no allocator.
+ *
+ * Same step and arguments as muon_step(), without a workspace: the scratch is
+ * a file-scope device array of MUON_STATIC_SCRATCH_BYTES inside the library,
+ * held on every device where the library is loaded until the process exits.
+ * The call allocates no device memory. The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture on that device.
+ *   - Returns MUON_ERR_WORKSPACE, before any device work, when the matrices
+ *     need more scratch than MUON_STATIC_SCRATCH_BYTES (see
+ *     muon_workspace_size for the amount).
+ *   - Each call writes its descriptor tables, including the counters that
+ *     must start at zero, into the array before its kernels run, so the
+ *     contents left by the previous call do not matter.
+ *   - All calls on a device share the one array: calls whose GPU work
+ *     overlaps (different streams, no ordering between them) race and give
+ *     wrong results. Order them on one stream or with events. */
+#define MUON_STATIC_SCRATCH_BYTES (64u << 20)
+
+MUON_API muon_status_t muon_step_static_scratch(const muon_param_t* params, int count, float lr,
+                                                float momentum, float weight_decay, float gamma,
+                                                int nesterov, const muon_ns_schedule_t* sched,
+                                                muon_precision_t prec, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

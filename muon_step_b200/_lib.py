@@ -18,13 +18,15 @@ MUON_ERR_TIMEOUT = 5
 MUON_NS_BF16 = 0
 MUON_NS_FP32 = 1
 
+MUON_STATIC_SCRATCH_BYTES = 64 << 20
+
 # every symbol include/muon_step.h declares
 EXPORTS = (
     "muon_plan_create", "muon_plan_create_ns", "muon_plan_workspace_size", "muon_plan_execute",
     "muon_plan_launches", "muon_plan_set_events", "muon_plan_flops", "muon_plan_destroy",
     "muon_workspace_size", "muon_step", "ns_workspace_size", "ns_orthogonalize",
     "muon_sync_status", "muon_status_string", "muon_abi_version", "muon_set_wait_limit_ns",
-    "muon_wait_probe",
+    "muon_wait_probe", "muon_step_static_scratch",
 )
 
 
@@ -85,6 +87,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_abi_version": (ctypes.c_int, []),
         "muon_set_wait_limit_ns": (None, [ctypes.c_uint64]),
         "muon_wait_probe": (st, [vp, ctypes.c_uint64, vp]),
+        "muon_step_static_scratch": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                          ctypes.c_float, ctypes.c_float, ctypes.c_int,
+                                          P(MuonNsSchedule), ctypes.c_int, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
