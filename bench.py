@@ -49,6 +49,7 @@ def parse_args():
     ap.add_argument("--config", default="batch64_1024")
     ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
     return ap.parse_args()
@@ -263,17 +264,41 @@ def main():
     torch.cuda.synchronize()
     assert ms.sync_status() == 0
 
-    # ---- timed region: device time with events, per-launch events inside
+    # ---- timed region: device time with events, per-launch events inside.
+    # By default the K steps (with their event records) are captured once in
+    # a CUDA graph and the timed region replays it.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(kinds))]
           for _ in range(args.steps)]
+    for k in range(args.steps):
+        for e in ev[k]:
+            e.record(stream)  # create the cudaEvent_t handles outside any capture
+    torch.cuda.synchronize()
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            graph.capture_begin()
+            for k in range(args.steps):
+                plan.set_events(ev[k], materialize=False)
+                plan.execute(ws, lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"],
+                             gamma=h["gamma"], nesterov=h["nesterov"], stream=cap)
+            graph.capture_end()
+        stream.wait_stream(cap)
+        plan.set_events(None)
+        torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t_start.record(stream)
-    for k in range(args.steps):
-        plan.set_events(ev[k])
-        step()
+    if graph is not None:
+        graph.replay()
+    else:
+        for k in range(args.steps):
+            plan.set_events(ev[k], materialize=False)
+            step()
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -390,11 +415,13 @@ def main():
             "kernels_share": {names[k]: v / tot_kernel for k, v in sorted(share.items())},
             "executed_tflops": (g_fl + p_fl + a_fl) / (ms_per_step / 1e3) / 1e12,
             "gpu_launches": len(kinds) * args.steps,
+            "cuda_graph": graph is not None,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    del graph
     del plan
     if world > 1:
         dist.barrier()

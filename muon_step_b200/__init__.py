@@ -110,15 +110,20 @@ class _PlanBase:
         _check(lib.muon_plan_launches(self._plan, ctypes.byref(n), kinds, n.value), "launches")
         return list(kinds)
 
-    def set_events(self, events: Optional[Sequence[torch.cuda.Event]]):
-        """Record events[2k] / events[2k+1] around launch k of every execute."""
+    def set_events(self, events: Optional[Sequence[torch.cuda.Event]], materialize=True):
+        """Record events[2k] / events[2k+1] around launch k of every execute.
+
+        torch creates an event's cudaEvent_t on its first record; pass
+        materialize=False only for events that have been recorded before (for
+        instance while capturing a CUDA graph)."""
         lib = _lib.load()
         if not events:
             _check(lib.muon_plan_set_events(self._plan, None, 0), "set_events")
             self._events = None
             return
-        for e in events:
-            e.record()  # materialise the underlying cudaEvent_t
+        if materialize:
+            for e in events:
+                e.record()
         handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib.muon_plan_set_events(self._plan, handles, len(events)), "set_events")
         self._events = list(events)
@@ -132,7 +137,9 @@ class _PlanBase:
 
     def _ws(self, workspace):
         if workspace is None:
-            workspace = self._own_ws = getattr(self, "_own_ws", None) or self.alloc_workspace()
+            if getattr(self, "_own_ws", None) is None:
+                self._own_ws = self.alloc_workspace()
+            workspace = self._own_ws
         if workspace.device.type != "cuda":
             raise TypeError("workspace must be a CUDA tensor")
         return workspace

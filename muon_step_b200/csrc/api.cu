@@ -70,20 +70,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor map over a group's [count][rows][ld] buffer, box {64, box_rows, 1},
-// 128-byte swizzle, zero fill outside [inner, rows, count].
-bool encode_bf16_3d(CUtensorMap* out, void* base, int64_t inner, int64_t rows, int64_t ld,
-                    int64_t count, int box_rows) {
+// 3-D tensor map over a group's [count][rows][ld] buffer, box {box0, box1, 1},
+// zero fill outside [inner, rows, count] on loads, clipping on stores.
+bool encode_3d(CUtensorMap* out, void* base, CUtensorMapDataType dtype, int elem_bytes, int64_t inner,
+               int64_t rows, int64_t ld, int64_t count, int box0, int box1,
+               CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(count)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2), static_cast<cuuint64_t>(rows * ld * 2)};
-  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * elem_bytes),
+                           static_cast<cuuint64_t>(rows * ld * elem_bytes)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(box1), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  return fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(out, dtype, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_bf16_3d(CUtensorMap* out, void* base, int64_t inner, int64_t rows, int64_t ld,
+                    int64_t count, int box0, int box1, CUtensorMapSwizzle swizzle) {
+  return encode_3d(out, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, rows, ld, count, box0, box1,
+                   swizzle);
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -108,8 +115,8 @@ struct muon_plan_s {
   int64_t ew_tiles = 0;
   int64_t stage_tiles[kNumKinds] = {0, 0, 0};
   double flops[kNumKinds] = {0, 0, 0};
-  size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_partial = 0, off_counter = 0,
-         off_scale = 0, desc_bytes = 0, ws_bytes = 0;
+  size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_mat_tmaps = 0, off_partial = 0,
+         off_counter = 0, off_scale = 0, desc_bytes = 0, ws_bytes = 0;
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -170,20 +177,21 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     gd.first_mat = static_cast<int32_t>(p->mats.size());
     double fl[kNumKinds] = {0, 0, 0};
     if (tc) {
-      const int64_t rb = cdiv(r, kBM);
-      int64_t syrk = 0;
+      // pair tiles of 256 x 256; the symmetric stages run those on or below
+      // the diagonal and keep the 128 x 128 blocks on or below it
+      const int64_t rb = cdiv(r, 128);
       for (int64_t i = 0; i < rb; ++i) {
-        syrk += i / 2 + 1;
-        const double rows = static_cast<double>(std::min<int64_t>(kBM, r - i * kBM));
-        for (int64_t bj = 0; bj <= i; ++bj) {  // computed and stored 128 x 128 blocks
-          const double cols = static_cast<double>(std::min<int64_t>(kBM, r - bj * kBM));
+        const double rows = static_cast<double>(std::min<int64_t>(128, r - i * 128));
+        for (int64_t bj = 0; bj <= i; ++bj) {
+          const double cols = static_cast<double>(std::min<int64_t>(128, r - bj * 128));
           fl[kGram] += 2.0 * rows * cols * static_cast<double>(c);
           fl[kPoly] += 2.0 * rows * cols * static_cast<double>(r);
         }
       }
-      gd.tiles_per_mat[kGram] = syrk;
-      gd.tiles_per_mat[kPoly] = syrk;
-      gd.tiles_per_mat[kApply] = rb * cdiv(c, kBN);
+      const int64_t pb = cdiv(r, kPairM);
+      gd.tiles_per_mat[kGram] = pb * (pb + 1) / 2;
+      gd.tiles_per_mat[kPoly] = gd.tiles_per_mat[kGram];
+      gd.tiles_per_mat[kApply] = pb * cdiv(c, kPairN);
     } else {
       gd.tiles_per_mat[kGram] = cdiv(r, kSBM) * cdiv(r, kSBN);
       gd.tiles_per_mat[kPoly] = gd.tiles_per_mat[kGram];
@@ -203,6 +211,11 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
       md.transposed = md.n > md.m ? 1 : 0;
       md.group = static_cast<int32_t>(g);
       md.index = static_cast<int32_t>(idx);
+      // the last step moves W and O by TMA when their rows are 16-byte aligned
+      const bool rows16 = (md.m % 4) == 0;
+      md.flags = 0;
+      if (md.W && rows16 && (reinterpret_cast<uintptr_t>(md.W) & 15) == 0) md.flags |= kMatWTma;
+      if (md.O && rows16 && (reinterpret_cast<uintptr_t>(md.O) & 15) == 0) md.flags |= kMatOTma;
       md.ew_tile_begin = ew_total;
       md.ew_tiles = cdiv(md.n, kEwRows) * cdiv(md.m, kEwCols);
       ew_total += md.ew_tiles;
@@ -220,6 +233,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + nm * sizeof(MatDesc), 256);
   p->off_tmaps = off;
   off = align_up(off + (tc ? ng * kTmPerGroup * sizeof(CUtensorMap) : 0), 256);
+  p->off_mat_tmaps = off;
+  off = align_up(off + (tc ? nm * kMtPerMat * sizeof(CUtensorMap) : 0), 256);
   p->off_partial = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
   p->off_counter = off;
@@ -270,14 +285,37 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
     for (size_t g = 0; g < p->groups.size(); ++g) {
       const GroupDesc& gd = p->groups[g];
       CUtensorMap* m = maps + g * kTmPerGroup;
+      const auto SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+      const auto SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
       const bool ok =
-          encode_bf16_3d(&m[kTmXb0K], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, kBM) &&
-          encode_bf16_3d(&m[kTmXb1K], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, kBM) &&
-          encode_bf16_3d(&m[kTmXb0MN], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 64) &&
-          encode_bf16_3d(&m[kTmXb1MN], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 64) &&
-          encode_bf16_3d(&m[kTmA], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, kBM) &&
-          encode_bf16_3d(&m[kTmB], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, kBM);
+          // operand maps (K blocks of 64 elements, 128-byte swizzle)
+          encode_bf16_3d(&m[kTmXb0K], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 64, 128, SW128) &&
+          encode_bf16_3d(&m[kTmXb1K], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 64, 128, SW128) &&
+          encode_bf16_3d(&m[kTmXb0MN], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 64, 64, SW128) &&
+          encode_bf16_3d(&m[kTmXb1MN], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 64, 64, SW128) &&
+          encode_bf16_3d(&m[kTmA], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 64, 128, SW128) &&
+          encode_bf16_3d(&m[kTmB], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 64, 128, SW128) &&
+          // epilogue maps (32 x 32 chunks)
+          encode_3d(&m[kTmXfE], base + gd.xf_off[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.c, gd.r,
+                    gd.ldc, gd.count, 32, 32, SW128) &&
+          encode_bf16_3d(&m[kTmXb0E], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
+          encode_bf16_3d(&m[kTmXb1E], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
+          encode_bf16_3d(&m[kTmAE], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64) &&
+          encode_bf16_3d(&m[kTmBE], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64);
       if (!ok) return MUON_ERR_CUDA;
+    }
+    auto* mmaps = reinterpret_cast<CUtensorMap*>(p->blob.data() + p->off_mat_tmaps);
+    for (size_t k = 0; k < p->mats.size(); ++k) {
+      const MatDesc& md = p->mats[k];
+      CUtensorMap* m = mmaps + k * kMtPerMat;
+      const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+      const auto SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+      if ((md.flags & kMatWTma) &&
+          !encode_3d(&m[kMtW], md.W, F32, 4, md.m, md.n, md.m, 1, 32, 32, SW128))
+        return MUON_ERR_CUDA;
+      if ((md.flags & kMatOTma) &&
+          !encode_3d(&m[kMtO], md.O, F32, 4, md.m, md.n, md.m, 1, 32, 32, SW128))
+        return MUON_ERR_CUDA;
     }
   }
   if (cudaMemcpyAsync(ws, p->blob.data(), p->desc_bytes, cudaMemcpyHostToDevice, stream) !=
@@ -288,11 +326,18 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
   return MUON_OK;
 }
 
+// Timing events around launches. Under stream capture the record must become
+// an external event node of the graph, or its timestamp cannot be read after
+// a replay.
 muon_status_t record(muon_plan_s* p, int slot, cudaStream_t stream) {
   if (p->events.empty()) return MUON_OK;
-  return cudaEventRecord(static_cast<cudaEvent_t>(p->events[slot]), stream) == cudaSuccess
-             ? MUON_OK
-             : MUON_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MUON_ERR_CUDA;
+  const cudaEvent_t ev = static_cast<cudaEvent_t>(p->events[slot]);
+  const cudaError_t e = (cap == cudaStreamCaptureStatusActive)
+                            ? cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal)
+                            : cudaEventRecord(ev, stream);
+  return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
 int launch_count(const muon_plan_s* p) { return 1 + 3 * p->steps; }
@@ -465,6 +510,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       sa.groups = groups;
       sa.mats = mats;
       sa.tmaps = ws + plan->off_tmaps;
+      sa.mat_tmaps = ws + plan->off_mat_tmaps;
       sa.ws = ws;
       sa.scale = scale;
       sa.err = err;
@@ -486,7 +532,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       cudaError_t e;
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
       if (tc) {
-        const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+        const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, sms / 2));
         e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, stream);
       } else {
         const int grid = static_cast<int>(std::min<int64_t>(tiles, 8LL * sms));

@@ -16,9 +16,9 @@ namespace muon {
 constexpr int kMaxGroups = 64;
 constexpr int kMaxSteps = 64;
 
-// tcgen05 tile shape: 128 x 256 output tiles, K blocks of 64 bf16 (128 B).
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+// tcgen05 tiles: 256 x 256 output tiles per CTA pair, K blocks of 64 bf16 (128 B).
+constexpr int kPairM = 256;
+constexpr int kPairN = 256;
 constexpr int kBK = 64;
 
 // fp32 validation tile shape.
@@ -32,6 +32,11 @@ constexpr int kEwCols = 128;
 
 enum StageKind : int { kGram = 0, kPoly = 1, kApply = 2, kNumKinds = 3 };
 
+// MatDesc.flags
+enum MatFlags : int { kMatWTma = 1, kMatOTma = 2 };
+// per-matrix tensor maps: fp32 {32, 32} boxes, 128-byte swizzle, over the caller's W and O
+enum MatTmapSlot : int { kMtW = 0, kMtO = 1, kMtPerMat = 2 };
+
 // tensor maps per group (bf16 mode)
 enum TmapSlot : int {
   kTmXb0K = 0,   // X bf16 buffer 0, box {64 cols, 128 rows}: K-major operand
@@ -40,7 +45,13 @@ enum TmapSlot : int {
   kTmXb1MN = 3,  // X bf16 buffer 1
   kTmA = 4,      // Gram matrix A, box {64, 128}
   kTmB = 5,      // polynomial B = bA + cA^2, box {64, 128}
-  kTmPerGroup = 6
+  // epilogue maps, box {32, 32}: loads and stores of one warp's 32 x 32 chunk
+  kTmXfE = 6,    // fp32 iterate, 128-byte swizzle
+  kTmXb0E = 7,   // bf16 iterate buffer 0, 64-byte swizzle
+  kTmXb1E = 8,   // bf16 iterate buffer 1, 64-byte swizzle
+  kTmAE = 9,     // A, 64-byte swizzle
+  kTmBE = 10,    // B, 64-byte swizzle
+  kTmPerGroup = 11
 };
 
 struct GroupDesc {
@@ -65,7 +76,7 @@ struct MatDesc {
   int32_t transposed;    // Newton-Schulz runs on the transpose (n > m)
   int32_t group;         // shape group
   int32_t index;         // index within the group
-  int32_t pad0;
+  int32_t flags;         // kMatWTma / kMatOTma: W / O reachable by TMA (16-byte rows)
   int64_t ew_tile_begin; // first elementwise tile of this matrix
   int64_t ew_tiles;      // number of elementwise tiles
 };
@@ -75,6 +86,7 @@ struct StageArgs {
   const GroupDesc* groups;
   const MatDesc* mats;
   const void* tmaps;      // CUtensorMap[ngroups][kTmPerGroup], 64-byte aligned
+  const void* mat_tmaps;  // CUtensorMap[nmats][kMtPerMat] (W / O of the last step)
   char* ws;               // workspace base
   const float* scale;     // per-matrix 1 / (||N||_F + eps)
   int* err;               // device error word

@@ -1,38 +1,49 @@
-// Newton-Schulz stages on the sm_100a tensor cores.
+// Newton-Schulz stages on the sm_100a tensor cores, one CTA pair per tile.
 //
-// One persistent, warp-specialised kernel per stage kind walks the output
-// tiles of every matrix of the plan (all shape groups, one launch):
+// One persistent, warp-specialised kernel per stage kind walks the 256 x 256
+// output tiles of every matrix of the plan (all shape groups, one launch).
+// CTAs run in clusters of two; the pair computes a tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16, bf16 x bf16 -> fp32):
+// each CTA holds 128 rows of the left operand and a 128-wide half of the
+// right operand in its shared memory, and 128 rows x 256 columns of the
+// accumulator in its TMEM. Per SM that is 32 KB of operands per 4.2 MFLOP,
+// two thirds of what a one-CTA 128 x 256 tile needs.
 //
-//   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of the two
-//              operands into a 4-deep shared-memory ring, one mbarrier per
-//              slot counting the bytes.
-//   warp 1     MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
-//              M = 128, N = 256, K = 16 per instruction, accumulating in
-//              TMEM; tcgen05.commit frees ring slots and hands finished
-//              accumulators to the epilogue. Two 256-column accumulators
-//              (all 512 TMEM columns) let the epilogue of one tile overlap
-//              the main loop of the next.
-//   warps 2-5  epilogue: tcgen05.ld of 32 columns at a time, one tile row
-//              per thread, fused arithmetic and stores.
+//   warp 0     TMA producer (both CTAs): 3-D tiled loads with 128-byte
+//              swizzle into a 4- or 5-deep ring; the bytes of both CTAs are
+//              counted on the pair leader's mbarrier.
+//   warp 1     TMEM allocation (both CTAs); MMA issue (leader only):
+//              tcgen05.commit multicasts slot releases and finished
+//              accumulators to both CTAs. Two 256-column accumulators let
+//              the epilogue of one tile overlap the main loop of the next.
+//   warps 2-5  epilogue (both CTAs): each warp owns 32 accumulator rows,
+//              reads 32 columns at a time from TMEM, stages results in
+//              swizzled shared memory and writes them with TMA tensor stores
+//              (whole lines, clipped at the matrix edge); inputs the
+//              epilogue needs (the fp32 iterate, the Gram tile, the weight)
+//              arrive by double-buffered TMA loads.
 //
 // Stages ("Ch 06 · Muon" §3 and §5 Algorithm 1, regrouped as
 // a X + (b A + c A^2) X with A = X X^T):
 //
-//   Gram   A = X X^T, symmetric: only tiles on or below the diagonal are
-//          computed (128 x 128 blocks, 256-wide tiles), each block stored
-//          and mirrored. Step one folds s^2 (X_0 = s N).
-//   Poly   B = b A + c A A^T (A symmetric); the epilogue reads A's tile.
-//          Lower tiles only, mirrored, like Gram.
-//   Apply  X' = a X + B X: B is the K-major left operand, the iterate X the
-//          MN-major right operand (row-major X read as K x N). The epilogue
-//          reads the fp32 iterate, writes the fp32 iterate and its bf16
-//          operand copy; on the last step it writes the update
-//          W <- W (1 - lr wd) - lr gamma sqrt(max(n, m)) X in the caller's
-//          orientation (and O' when requested).
+//   Gram       A = X X^T. Symmetric: only pair tiles on or below the diagonal
+//              run; each 128 x 128 block on or below the diagonal is stored
+//              and, below the diagonal, mirrored. Step one folds s^2
+//              (X_0 = s N).
+//   Poly       B = b A + c A A^T (A symmetric), same tiling as Gram.
+//   Apply      X' = a X + B X: B is the K-major left operand, the iterate X
+//              the MN-major right operand (row-major X read as K x N). Step
+//              one folds s.
+//   ApplyLast  the last step's Apply: O' = a X + B X, then the update of
+//              "Muon 优化器完全拆解…", Algorithm 1 steps four and five,
+//              W <- W (1 - lr wd) - lr gamma sqrt(max(n, m)) O', in the
+//              caller's orientation (and O' when requested). W and O move by
+//              TMA when their rows are 16-byte aligned, else by coalesced
+//              plain loads and stores.
 //
-// Every spin-wait is bounded; on expiry the kernel sets the error word,
-// stops issuing work, waits (bounded) for copies and MMAs already in
-// flight, frees TMEM and returns.
+// Every spin-wait is bounded; on expiry the kernel raises the error word and
+// an abort flag in both CTAs, stops issuing work, drains what is in flight,
+// frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -43,96 +54,153 @@ namespace muon {
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK * 2;             // 16 KB
-constexpr int kBBytes = kBN * kBK * 2;             // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;     // 48 KB
-constexpr int kTmemCols = 512;                     // two 256-column accumulators
-constexpr int kTmapBytes = 128;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr size_t kBarrierBytes = 256;
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kBarrierBytes;
+constexpr int kApplyLast = 3;  // kernel kind beyond StageKind: the last Apply
 
-constexpr uint32_t kIdescKK = ptx::idesc_bf16(kBM, kBN, 0, 0);   // both K-major
-constexpr uint32_t kIdescKMN = ptx::idesc_bf16(kBM, kBN, 0, 1);  // B MN-major
+constexpr int kHalf = 128;                        // rows of each operand half held by one CTA
+constexpr int kABytes = kHalf * kBK * 2;          // 16 KB
+constexpr int kBBytes = kHalf * kBK * 2;          // 16 KB
+constexpr int kStageBytes = kABytes + kBBytes;    // 32 KB
+constexpr uint32_t kPairTx = 2 * kStageBytes;     // bytes both CTAs land per ring slot
+constexpr int kPairTile = 256;
+constexpr int kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kEpiF32 = 32 * 32 * 4;              // fp32 32 x 32, 128-byte swizzle
+constexpr int kEpiB16 = 32 * 32 * 2;              // bf16 32 x 32, 64-byte swizzle
+constexpr size_t kBarrierBytes = 256;
+constexpr int kTmapBytes = 128;
+
+// Per-kind layout. Epilogue staging slot (two per warp):
+//   Gram / Poly  [bf16 A in (Poly) | bf16 out | bf16 mirror out]   6 KB
+//   Apply        [fp32 iterate in / out | bf16 iterate out]         6 KB
+//   ApplyLast    [fp32 iterate in / O out | fp32 W in / out]        8 KB
+template <int KIND>
+struct Cfg {
+  static constexpr int kStages = (KIND == kApplyLast) ? 4 : 5;
+  static constexpr int kSlot = (KIND == kApplyLast) ? 2 * kEpiF32 : kEpiF32 + kEpiB16;
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kSlot;
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarrierBytes;
+  static constexpr bool kApplyLike = (KIND == kApply || KIND == kApplyLast);
+  static constexpr int kTiles = kApplyLike ? kApply : KIND;  // which tile tables to walk
+};
+
+constexpr int kOffSymOut = kEpiB16;
+constexpr int kOffSymMirror = 2 * kEpiB16;
+constexpr int kOffApplyOut16 = kEpiF32;
+constexpr int kOffLastW = kEpiF32;
+
+constexpr uint32_t kIdescKK = ptx::idesc_bf16(kPairTile, kPairTile, 0, 0);   // both K-major
+constexpr uint32_t kIdescKMN = ptx::idesc_bf16(kPairTile, kPairTile, 0, 1);  // B MN-major
 
 struct TileCoord {
   int g;
   int64_t b;    // matrix within the group
-  int i;        // 128-row block
-  int j;        // 256-column tile
+  int I, J;     // 256-row block, 256-column block
   int kblocks;  // K / 64, rounded up
 };
 
-// Lower-triangle tile enumeration for the symmetric stages: row block i
-// (128 rows) has tiles j = 0 .. floor(i / 2) (256 columns each). Row pair p
-// (rows 2p, 2p + 1) holds 2 (p + 1) tiles; the first p pairs hold p (p + 1).
-__device__ __forceinline__ void syrk_tile(int64_t u, int& i, int& j) {
-  int64_t p = static_cast<int64_t>((sqrt(4.0 * static_cast<double>(u) + 1.0) - 1.0) * 0.5);
-  while (p * (p + 1) > u) --p;
-  while ((p + 1) * (p + 2) <= u) ++p;
-  const int64_t off = u - p * (p + 1);
-  if (off <= p) {
-    i = static_cast<int>(2 * p);
-    j = static_cast<int>(off);
-  } else {
-    i = static_cast<int>(2 * p + 1);
-    j = static_cast<int>(off - (p + 1));
-  }
+// Lower-triangle pair tiles of the symmetric stages: (I, J) with J <= I,
+// row-major: u = I (I + 1) / 2 + J.
+__device__ __forceinline__ void lower_tile(int64_t u, int& I, int& J) {
+  int64_t i = static_cast<int64_t>((sqrt(8.0 * static_cast<double>(u) + 1.0) - 1.0) * 0.5);
+  while (i * (i + 1) / 2 > u) --i;
+  while ((i + 1) * (i + 2) / 2 <= u) ++i;
+  I = static_cast<int>(i);
+  J = static_cast<int>(u - i * (i + 1) / 2);
 }
 
 template <int KIND>
 __device__ __forceinline__ TileCoord decode_tile(const StageArgs& a, int64_t t) {
+  constexpr int T = Cfg<KIND>::kTiles;
   TileCoord tc;
-  tc.g = stage_group<KIND>(a, t);
+  tc.g = stage_group<T>(a, t);
   const GroupDesc& gd = a.groups[tc.g];
-  const int64_t local = t - gd.tile_base[KIND];
-  const int64_t per = gd.tiles_per_mat[KIND];
+  const int64_t local = t - gd.tile_base[T];
+  const int64_t per = gd.tiles_per_mat[T];
   tc.b = local / per;
   const int64_t u = local % per;
-  if (KIND == kApply) {
-    const int64_t rb = (gd.r + kBM - 1) / kBM;
-    tc.i = static_cast<int>(u % rb);
-    tc.j = static_cast<int>(u / rb);
+  if (T == kApply) {
+    const int64_t rb = (gd.r + kPairTile - 1) / kPairTile;
+    tc.I = static_cast<int>(u % rb);
+    tc.J = static_cast<int>(u / rb);
     tc.kblocks = (gd.r + kBK - 1) / kBK;
   } else {
-    syrk_tile(u, tc.i, tc.j);
-    tc.kblocks = ((KIND == kGram ? gd.c : gd.r) + kBK - 1) / kBK;
+    lower_tile(u, tc.I, tc.J);
+    tc.kblocks = ((T == kGram ? gd.c : gd.r) + kBK - 1) / kBK;
   }
   return tc;
 }
 
 __device__ __forceinline__ const void* tmap(const StageArgs& a, int g, int slot) {
-  return static_cast<const char*>(a.tmaps) + (static_cast<int64_t>(g) * kTmPerGroup + slot) * kTmapBytes;
+  return static_cast<const char*>(a.tmaps) +
+         (static_cast<int64_t>(g) * kTmPerGroup + slot) * kTmapBytes;
 }
 
-__device__ __forceinline__ void raise_abort(const StageArgs& a, volatile int* abort_flag) {
-  *abort_flag = 1;
-  atomicOr(a.err, kErrTimeout);
+__device__ __forceinline__ const void* mat_tmap(const StageArgs& a, int mat, int slot) {
+  return static_cast<const char*>(a.mat_tmaps) +
+         (static_cast<int64_t>(mat) * kMtPerMat + slot) * kTmapBytes;
 }
 
 struct alignas(16) Bf16x8 {
   __nv_bfloat162 v[4];
 };
 
-// -------------------------------------------------------------- epilogues
+// Byte offsets inside the swizzled staging tiles (buffers aligned to the
+// swizzle period): 128-byte rows of fp32 (16-byte chunk q of row r lands at
+// chunk q ^ (r % 8)); 64-byte rows of bf16 (chunk q ^ ((r / 2) % 4)).
+__device__ __forceinline__ int sw128_chunk(int row, int q) { return row * 128 + ((q ^ (row & 7)) << 4); }
+__device__ __forceinline__ int sw64_chunk(int row, int q) { return row * 64 + ((q ^ ((row >> 1) & 3)) << 4); }
+// fp32 element (row, col) of a 32 x 32 tile with 128-byte swizzle
+__device__ __forceinline__ int sw128_f32(int row, int col) { return sw128_chunk(row, col >> 2) + ((col & 3) << 2); }
 
-// Gram / Poly: 32 columns of one row of a lower (or diagonal) 128 x 128 block.
+// -------------------------------------------------------------- shared state
+
+struct Smem {
+  uint8_t* ring;   // stages x (A half | B half)
+  uint8_t* epi;    // kEpiWarps x 2 slots
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* drain;
+  uint64_t* eload;  // kEpiWarps x 2
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+};
+
+template <int KIND>
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.ring = base;
+  s.epi = base + Cfg<KIND>::kStages * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.epi + Cfg<KIND>::kEpiBytes);
+  s.full = bars;
+  s.empty = s.full + Cfg<KIND>::kStages;
+  s.tfull = s.empty + Cfg<KIND>::kStages;
+  s.tempty = s.tfull + 2;
+  s.drain = s.tempty + 2;
+  s.eload = s.drain + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + 2 * kEpiWarps);
+  s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
+  return s;
+}
+
+// Raise the abort flag in both CTAs of the pair and the device error word.
+__device__ __forceinline__ void raise_abort(const StageArgs& a, const Smem& s) {
+  const uint32_t local = ptx::smem_u32(const_cast<int*>(s.abort_flag));
+  ptx::st_cluster_u32(ptx::mapa_shared(local, 0), 1u);
+  ptx::st_cluster_u32(ptx::mapa_shared(local, 1), 1u);
+  atomicOr(a.err, kErrTimeout);
+}
+
+// -------------------------------------------------------------- epilogue pieces
+
+// Gram / Poly: one warp's 32 x 32 chunk of a block on or below the diagonal.
 template <int KIND>
 __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const GroupDesc& gd,
-                                              const TileCoord& tc, int trow, int ch,
-                                              const float (&v)[32]) {
-  const int bj = 2 * tc.j + (ch >> 2);
-  if (bj > tc.i) return;  // block above the diagonal: its mirror is stored elsewhere
-  const int64_t r = gd.r, ldr = gd.ldr;
-  const int64_t row = static_cast<int64_t>(tc.i) * kBM + trow;
-  const int64_t col0 = static_cast<int64_t>(tc.j) * kBN + ch * 32;
-  if (row >= r || col0 >= r) return;
-  const int ncol = static_cast<int>(r - col0 < 32 ? r - col0 : 32);
-  const int64_t moff = tc.b * r * ldr;
-  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.ws + (KIND == kGram ? gd.a_off : gd.b_off)) + moff;
-
+                                              const TileCoord& tc, int row0, int col0, bool mirror,
+                                              uint8_t* slot, const float (&v)[32], int lane) {
   float out[32];
   if (KIND == kGram) {
     float s2 = 1.f;
@@ -143,203 +211,280 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const GroupDes
 #pragma unroll
     for (int e = 0; e < 32; ++e) out[e] = s2 * v[e];
   } else {
-    const __nv_bfloat16* Asrc = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.a_off) + moff + row * ldr + col0;
-    if (ncol == 32) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const Bf16x8 p = *reinterpret_cast<const Bf16x8*>(Asrc + 8 * q);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float2 f = __bfloat1622float2(p.v[h]);
-          out[8 * q + 2 * h] = fmaf(a.b, f.x, a.c * v[8 * q + 2 * h]);
-          out[8 * q + 2 * h + 1] = fmaf(a.b, f.y, a.c * v[8 * q + 2 * h + 1]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        out[e] = (e < ncol) ? fmaf(a.b, __bfloat162float(Asrc[e]), a.c * v[e]) : 0.f;
-    }
-  }
-
-  __nv_bfloat16* drow = dst + row * ldr + col0;
-  if (ncol == 32) {
+    // the A chunk, bf16 with 64-byte swizzle, in the slot's input area
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      Bf16x8 p;
+      const Bf16x8 p = *reinterpret_cast<const Bf16x8*>(slot + sw64_chunk(lane, q));
 #pragma unroll
-      for (int h = 0; h < 4; ++h) p.v[h] = __floats2bfloat162_rn(out[8 * q + 2 * h], out[8 * q + 2 * h + 1]);
-      *reinterpret_cast<Bf16x8*>(drow + 8 * q) = p;
+      for (int h = 0; h < 4; ++h) {
+        const float2 f = __bfloat1622float2(p.v[h]);
+        out[8 * q + 2 * h] = fmaf(a.b, f.x, a.c * v[8 * q + 2 * h]);
+        out[8 * q + 2 * h + 1] = fmaf(a.b, f.y, a.c * v[8 * q + 2 * h + 1]);
+      }
     }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (e < ncol) drow[e] = __float2bfloat16_rn(out[e]);
   }
-  if (bj < tc.i) {
-    // mirror: lanes hold consecutive rows, so each store is 64 contiguous bytes
+  uint8_t* st_direct = slot + kOffSymOut;
+  uint8_t* st_mirror = slot + kOffSymMirror;
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (e < ncol) dst[(col0 + e) * ldr + row] = __float2bfloat16_rn(out[e]);
+  for (int q = 0; q < 4; ++q) {
+    Bf16x8 p;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) p.v[h] = __floats2bfloat162_rn(out[8 * q + 2 * h], out[8 * q + 2 * h + 1]);
+    *reinterpret_cast<Bf16x8*>(st_direct + sw64_chunk(lane, q)) = p;
+  }
+  if (mirror) {
+    // transposed chunk: row e of the mirror holds column e of this chunk
+    __nv_bfloat16* m16 = reinterpret_cast<__nv_bfloat16*>(st_mirror);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int off = sw64_chunk(e, lane >> 3) + (lane & 7) * 2;
+      m16[off >> 1] = __float2bfloat16_rn(out[e]);
+    }
+  }
+  ptx::fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    const void* tm = tmap(a, tc.g, KIND == kGram ? kTmAE : kTmBE);
+    ptx::tma_store_3d(tm, st_direct, col0, row0, static_cast<int>(tc.b));
+    if (mirror) ptx::tma_store_3d(tm, st_mirror, row0, col0, static_cast<int>(tc.b));
   }
 }
 
-// Apply: X' = alpha (a X + acc) for 32 columns of one row.
-__device__ __forceinline__ void epi_apply(const StageArgs& a, const GroupDesc& gd,
-                                          const TileCoord& tc, int trow, int ch,
-                                          const float (&v)[32]) {
-  const int64_t r = gd.r, c = gd.c, ldc = gd.ldc;
-  const int64_t row = static_cast<int64_t>(tc.i) * kBM + trow;
-  const int64_t col0 = static_cast<int64_t>(tc.j) * kBN + ch * 32;
-  if (row >= r || col0 >= c) return;
-  const int ncol = static_cast<int>(c - col0 < 32 ? c - col0 : 32);
+// X' (or O') = alpha (a X + acc) for one warp's 32 x 32 chunk; X from the
+// slot's fp32 input area.
+__device__ __forceinline__ void apply_values(const StageArgs& a, float alpha, const uint8_t* slot,
+                                             const float (&v)[32], int lane, float (&x)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 p = *reinterpret_cast<const float4*>(slot + sw128_chunk(lane, q));
+    x[4 * q + 0] = alpha * fmaf(a.a, p.x, v[4 * q + 0]);
+    x[4 * q + 1] = alpha * fmaf(a.a, p.y, v[4 * q + 1]);
+    x[4 * q + 2] = alpha * fmaf(a.a, p.z, v[4 * q + 2]);
+    x[4 * q + 3] = alpha * fmaf(a.a, p.w, v[4 * q + 3]);
+  }
+}
+
+// Apply: write the new fp32 iterate and its bf16 operand copy.
+__device__ __forceinline__ void epi_apply(const StageArgs& a, const GroupDesc& gd, const TileCoord& tc,
+                                          int row0, int col0, uint8_t* slot, const float (&v)[32],
+                                          int lane) {
   const int mat = gd.first_mat + static_cast<int>(tc.b);
   const float alpha = a.first ? a.scale[mat] : 1.f;
-  float* xf = reinterpret_cast<float*>(a.ws + gd.xf_off[0]) + tc.b * r * ldc + row * ldc + col0;
-
   float x[32];
-  if (ncol == 32) {
+  apply_values(a, alpha, slot, v, lane, x);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 p = *reinterpret_cast<const float4*>(xf + 4 * q);
-      x[4 * q + 0] = alpha * fmaf(a.a, p.x, v[4 * q + 0]);
-      x[4 * q + 1] = alpha * fmaf(a.a, p.y, v[4 * q + 1]);
-      x[4 * q + 2] = alpha * fmaf(a.a, p.z, v[4 * q + 2]);
-      x[4 * q + 3] = alpha * fmaf(a.a, p.w, v[4 * q + 3]);
-    }
-  } else {
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(slot + sw128_chunk(lane, q)) =
+        make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+  uint8_t* st16 = slot + kOffApplyOut16;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) x[e] = (e < ncol) ? alpha * fmaf(a.a, xf[e], v[e]) : 0.f;
+  for (int q = 0; q < 4; ++q) {
+    Bf16x8 p;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) p.v[h] = __floats2bfloat162_rn(x[8 * q + 2 * h], x[8 * q + 2 * h + 1]);
+    *reinterpret_cast<Bf16x8*>(st16 + sw64_chunk(lane, q)) = p;
   }
+  ptx::fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    ptx::tma_store_3d(tmap(a, tc.g, kTmXfE), slot, col0, row0, static_cast<int>(tc.b));
+    ptx::tma_store_3d(tmap(a, tc.g, a.xsrc ? kTmXb0E : kTmXb1E), st16, col0, row0,
+                      static_cast<int>(tc.b));
+  }
+}
 
-  if (!a.last) {
-    __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xb_off[a.xsrc ^ 1]) + tc.b * r * ldc + row * ldc + col0;
-    if (ncol == 32) {
+// Whether the last step moves this matrix's W and O by TMA.
+__device__ __forceinline__ bool last_by_tma(const MatDesc& md) {
+  return (!md.W || (md.flags & kMatWTma)) && (!md.O || (md.flags & kMatOTma));
+}
+
+// Caller coordinates (x = column, y = row) of the chunk at iterate (row0, col0).
+__device__ __forceinline__ void caller_xy(const MatDesc& md, int row0, int col0, int& x, int& y) {
+  x = md.transposed ? row0 : col0;
+  y = md.transposed ? col0 : row0;
+}
+
+// ApplyLast: O' and the update, W <- W keep - step O', in the caller's
+// orientation. With TMA the W chunk is in the slot's second area, in the
+// caller's orientation (transposed relative to the iterate when n > m).
+__device__ __forceinline__ void epi_apply_last(const StageArgs& a, const GroupDesc& gd,
+                                               const TileCoord& tc, int row0, int col0, uint8_t* slot,
+                                               const float (&v)[32], int lane) {
+  const int mat = gd.first_mat + static_cast<int>(tc.b);
+  const float alpha = a.first ? a.scale[mat] : 1.f;
+  float x[32];
+  apply_values(a, alpha, slot, v, lane, x);
+  const MatDesc& md = a.mats[mat];
+  const UpdateConsts uc = update_consts(a, gd.c);
+  const bool tr = md.transposed != 0;
+
+  if (last_by_tma(md)) {
+    // element (iterate row lane, col e) sits at (lane, e), or at (e, lane) when transposed
+    if (md.W) {
+      uint8_t* Ws = slot + kOffLastW;
+      if (!tr) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(xf + 4 * q) = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        Bf16x8 p;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) p.v[h] = __floats2bfloat162_rn(x[8 * q + 2 * h], x[8 * q + 2 * h + 1]);
-        *reinterpret_cast<Bf16x8*>(xb + 8 * q) = p;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (e < ncol) {
-          xf[e] = x[e];
-          xb[e] = __float2bfloat16_rn(x[e]);
+        for (int q = 0; q < 8; ++q) {
+          float4* p = reinterpret_cast<float4*>(Ws + sw128_chunk(lane, q));
+          float4 w = *p;
+          w.x = fmaf(w.x, uc.keep, -uc.step * x[4 * q + 0]);
+          w.y = fmaf(w.y, uc.keep, -uc.step * x[4 * q + 1]);
+          w.z = fmaf(w.z, uc.keep, -uc.step * x[4 * q + 2]);
+          w.w = fmaf(w.w, uc.keep, -uc.step * x[4 * q + 3]);
+          *p = w;
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float* p = reinterpret_cast<float*>(Ws + sw128_f32(e, lane));
+          *p = fmaf(*p, uc.keep, -uc.step * x[e]);
+        }
+      }
+    }
+    if (md.O) {
+      __syncwarp();  // every lane has read its iterate values: the area takes O'
+      if (!tr) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4*>(slot + sw128_chunk(lane, q)) =
+              make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) *reinterpret_cast<float*>(slot + sw128_f32(e, lane)) = x[e];
+      }
+    }
+    ptx::fence_async_shared();
+    __syncwarp();
+    if (lane == 0) {
+      int cx, cy;
+      caller_xy(md, row0, col0, cx, cy);
+      if (md.W) ptx::tma_store_3d(mat_tmap(a, mat, kMtW), slot + kOffLastW, cx, cy, 0);
+      if (md.O) ptx::tma_store_3d(mat_tmap(a, mat, kMtO), slot, cx, cy, 0);
     }
     return;
   }
 
-  // last step: the update, in the caller's orientation
-  const MatDesc& md = a.mats[mat];
-  const UpdateConsts uc = update_consts(a, static_cast<int>(c));
-  if (!md.transposed && ncol == 32 && (md.m & 3) == 0 &&
-      ((reinterpret_cast<uintptr_t>(md.W) | reinterpret_cast<uintptr_t>(md.O)) & 15) == 0) {
-    const int64_t base = row * md.m + col0;
+  // Plain loads and stores (rows not 16-byte aligned).
+  const int mrows = (gd.r - row0) < 32 ? (gd.r - row0) : 32;
+  const int ncol = (gd.c - col0) < 32 ? (gd.c - col0) : 32;
+  if (tr) {
+    // caller element (col, row): for each column the lanes (rows) hit consecutive addresses
+    if (lane < mrows) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 o4 = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-      if (md.O) *reinterpret_cast<float4*>(md.O + base + 4 * q) = o4;
-      if (md.W) {
-        float4 w = *reinterpret_cast<const float4*>(md.W + base + 4 * q);
-        w.x = fmaf(w.x, uc.keep, -uc.step * o4.x);
-        w.y = fmaf(w.y, uc.keep, -uc.step * o4.y);
-        w.z = fmaf(w.z, uc.keep, -uc.step * o4.z);
-        w.w = fmaf(w.w, uc.keep, -uc.step * o4.w);
-        *reinterpret_cast<float4*>(md.W + base + 4 * q) = w;
-      }
+      for (int e = 0; e < 32; ++e)
+        if (e < ncol) write_update(md, uc, row0 + lane, col0 + e, x[e]);
     }
-  } else {
-    // transposed: for each column, the warp's lanes write consecutive addresses
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (e < ncol) write_update(md, uc, row, col0 + e, x[e]);
+    return;
   }
+  // Row-major caller matrix: move O' to "lane = column" layout through a
+  // 32 x 32 transpose in shared memory (word (r, c) at r * 32 + (c ^ r):
+  // conflict-free both ways); then every global access of the warp is one
+  // contiguous row segment, all 32 rows' loads in flight at once. The slot's
+  // second area is unused on this path.
+  float* T = reinterpret_cast<float*>(slot + kOffLastW);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) T[lane * 32 + (e ^ lane)] = x[e];
+  __syncwarp();
+  float xc[32];
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) xc[rr] = T[rr * 32 + (lane ^ rr)];
+  const bool col_ok = lane < ncol;
+  float* Wp = md.W ? md.W + static_cast<int64_t>(row0) * md.m + col0 + lane : nullptr;
+  float* Op = md.O ? md.O + static_cast<int64_t>(row0) * md.m + col0 + lane : nullptr;
+  if (Op) {
+#pragma unroll
+    for (int rr = 0; rr < 32; ++rr)
+      if (col_ok && rr < mrows) Op[static_cast<int64_t>(rr) * md.m] = xc[rr];
+  }
+  if (Wp) {
+    float w[32];
+#pragma unroll
+    for (int rr = 0; rr < 32; ++rr) w[rr] = (col_ok && rr < mrows) ? Wp[static_cast<int64_t>(rr) * md.m] : 0.f;
+#pragma unroll
+    for (int rr = 0; rr < 32; ++rr)
+      if (col_ok && rr < mrows) Wp[static_cast<int64_t>(rr) * md.m] = fmaf(w[rr], uc.keep, -uc.step * xc[rr]);
+  }
+  // a later TMA load may overwrite this slot: order these accesses before it
+  ptx::fence_async_shared();
+  __syncwarp();
 }
 
 // -------------------------------------------------------------- kernel
 
 template <int KIND>
-__global__ void __launch_bounds__(kThreads, 1) stage_tc_kernel(const __grid_constant__ StageArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    stage_tc_kernel(const __grid_constant__ StageArgs a) {
+  using C = Cfg<KIND>;
+  constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
+  const Smem s = carve<KIND>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int64_t pair = blockIdx.x >> 1;
+  const int64_t npairs = gridDim.x >> 1;
+  const uint64_t limit = a.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&empty[s], 1);
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&s.full[i], 1);
+      ptx::mbar_init(&s.empty[i], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&tfull[s], 1);
-      ptx::mbar_init(&tempty[s], kEpiThreads);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&s.tfull[i], 1);
+      ptx::mbar_init(&s.tempty[i], 2 * kEpiWarps);
     }
-    ptx::mbar_init(drain, 1);
-    *abort_flag = 0;
+    ptx::mbar_init(s.drain, 1);
+    for (int i = 0; i < 2 * kEpiWarps; ++i) ptx::mbar_init(&s.eload[i], 1);
+    *s.abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(s.tmem_slot, kTmemCols);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();  // barriers of both CTAs initialised before any remote use
   ptx::tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const uint64_t limit = a.wait_limit_ns;
+  const uint32_t tmem_base = *s.tmem_slot;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- producer
     for (int g = 0; g < a.ngroups; ++g)
-      for (int s = 0; s < kTmPerGroup; ++s) {
-        ptx::fence_tmap_acquire(tmap(a, g, s));
-        ptx::prefetch_tmap(tmap(a, g, s));
+      for (int k = 0; k < kTmPerGroup; ++k) {
+        ptx::fence_tmap_acquire(tmap(a, g, k));
+        ptx::prefetch_tmap(tmap(a, g, k));
       }
+    uint32_t leader_full[kStages];
+    for (int i = 0; i < kStages; ++i) leader_full[i] = ptx::mapa_shared(ptx::smem_u32(&s.full[i]), 0);
     uint32_t stage = 0, phase = 0;
-    uint32_t armed = 0, armed_phase = 0;  // bit s: slot s armed; its last armed parity
     bool ok = true;
-    for (int64_t t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
+    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
       const int bz = static_cast<int>(tc.b);
       for (int kb = 0; kb < tc.kblocks; ++kb) {
-        if (!ptx::mbar_wait(&empty[stage], phase ^ 1, limit, abort_flag)) {
-          raise_abort(a, abort_flag);
+        if (!ptx::mbar_wait(&s.empty[stage], phase ^ 1, limit, s.abort_flag)) {
+          raise_abort(a, s);
           ok = false;
           break;
         }
-        uint8_t* sa = smem + stage * kStageBytes;
+        uint8_t* sa = s.ring + stage * kStageBytes;
         uint8_t* sb = sa + kABytes;
-        ptx::mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        armed |= 1u << stage;
-        armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+        if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], kPairTx);
         const int k0 = kb * kBK;
-        if (KIND == kApply) {
-          ptx::tma_load_3d(sa, tmap(a, tc.g, kTmB), &full[stage], k0, tc.i * kBM, bz);
+        if (C::kApplyLike) {
+          ptx::tma_load_3d_pair(sa, tmap(a, tc.g, kTmB), leader_full[stage], k0,
+                                tc.I * kPairTile + rank * kHalf, bz);
           const void* tx = tmap(a, tc.g, a.xsrc ? kTmXb1MN : kTmXb0MN);
 #pragma unroll
-          for (int q = 0; q < kBN / 64; ++q)
-            ptx::tma_load_3d(sb + q * (64 * kBK * 2), tx, &full[stage], tc.j * kBN + q * 64, k0, bz);
+          for (int q = 0; q < kHalf / 64; ++q)
+            ptx::tma_load_3d_pair(sb + q * (64 * kBK * 2), tx, leader_full[stage],
+                                  tc.J * kPairTile + rank * kHalf + q * 64, k0, bz);
         } else {
           const void* tm = (KIND == kGram) ? tmap(a, tc.g, a.xsrc ? kTmXb1K : kTmXb0K)
                                            : tmap(a, tc.g, kTmA);
-          ptx::tma_load_3d(sa, tm, &full[stage], k0, tc.i * kBM, bz);
-          ptx::tma_load_3d(sb, tm, &full[stage], k0, tc.j * kBN, bz);
-          ptx::tma_load_3d(sb + kABytes, tm, &full[stage], k0, tc.j * kBN + kBM, bz);
+          ptx::tma_load_3d_pair(sa, tm, leader_full[stage], k0, tc.I * kPairTile + rank * kHalf, bz);
+          ptx::tma_load_3d_pair(sb, tm, leader_full[stage], k0, tc.J * kPairTile + rank * kHalf, bz);
         }
         if (++stage == kStages) {
           stage = 0;
@@ -348,128 +493,204 @@ __global__ void __launch_bounds__(kThreads, 1) stage_tc_kernel(const __grid_cons
       }
     }
     if (!ok) {
-      // let the copies already issued land before the CTA exits
-      volatile int never = 0;
-      for (int s = 0; s < kStages; ++s)
-        if (armed & (1u << s)) ptx::mbar_wait(&full[s], (armed_phase >> s) & 1u, limit, &never);
+      // give copies already issued time to land before the pair exits
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (ptx::globaltimer_ns() - t0 < 20000) {
+      }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    const uint32_t idesc = (KIND == kApply) ? kIdescKMN : kIdescKK;
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------------------------------------------------- MMA issuer (pair leader)
+    const uint32_t idesc = C::kApplyLike ? kIdescKMN : kIdescKK;
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
     bool ok = true;
     bool issued = false;
-    for (int64_t t = blockIdx.x; ok && t < a.total_tiles; t += gridDim.x) {
+    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
-      if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1, limit, abort_flag)) {
-        raise_abort(a, abort_flag);
+      if (!ptx::mbar_wait(&s.tempty[acc], acc_phase ^ 1, limit, s.abort_flag)) {
+        raise_abort(a, s);
         ok = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t d = tmem_base + acc * kBN;
+      const uint32_t d = tmem_base + acc * kPairTile;
       for (int kb = 0; kb < tc.kblocks; ++kb) {
-        if (!ptx::mbar_wait(&full[stage], phase, limit, abort_flag)) {
-          raise_abort(a, abort_flag);
+        if (!ptx::mbar_wait(&s.full[stage], phase, limit, s.abort_flag)) {
+          raise_abort(a, s);
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t sa = ptx::smem_u32(smem + stage * kStageBytes);
+        const uint32_t sa = ptx::smem_u32(s.ring + stage * kStageBytes);
         const uint32_t sb = sa + kABytes;
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t ad = ptx::desc_sw128(sa + k * 32, 16, 1024);
-          const uint64_t bd = (KIND == kApply) ? ptx::desc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
-                                               : ptx::desc_sw128(sb + k * 32, 16, 1024);
-          ptx::umma_bf16(d, ad, bd, idesc, (kb | k) != 0);
+          const uint64_t bd = C::kApplyLike ? ptx::desc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
+                                            : ptx::desc_sw128(sb + k * 32, 16, 1024);
+          ptx::umma_bf16_pair(d, ad, bd, idesc, (kb | k) != 0);
         }
         issued = true;
-        ptx::umma_commit(&empty[stage]);
+        ptx::umma_commit_pair(&s.empty[stage]);
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      ptx::umma_commit(&tfull[acc]);
+      ptx::umma_commit_pair(&s.tfull[acc]);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
     if (!ok && issued) {
-      // wait for the MMAs in flight before TMEM is released
+      // let the MMAs in flight finish before TMEM is released
       volatile int never = 0;
-      ptx::umma_commit(drain);
-      ptx::mbar_wait(drain, 0, limit, &never);
+      ptx::umma_commit_pair_self(s.drain);
+      ptx::mbar_wait(s.drain, 0, limit, &never);
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------- epilogue
-    const int lane_base = (warp & 3) * 32;  // TMEM lanes this warp may read
-    const int trow = lane_base + lane;
+    const int ew = warp - 2;
+    const int quarter = warp & 3;  // TMEM lanes this warp may read: 32 * quarter ...
+    uint8_t* slots = s.epi + ew * 2 * C::kSlot;
+    uint64_t* eload = s.eload + 2 * ew;
+    uint32_t eload_phase[2] = {0u, 0u};
+    uint32_t leader_tempty[2];
+    for (int i = 0; i < 2; ++i) leader_tempty[i] = ptx::mapa_shared(ptx::smem_u32(&s.tempty[i]), 0);
+    constexpr bool kInput = (KIND != kGram);
     uint32_t acc = 0, acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
+    bool ok = true;
+    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
-      if (!ptx::mbar_wait(&tfull[acc], acc_phase, limit, abort_flag)) {
-        raise_abort(a, abort_flag);
-        break;
+      const GroupDesc& gd = a.groups[tc.g];
+      const int row0 = tc.I * kPairTile + static_cast<int>(rank) * kHalf + quarter * 32;
+      const int bi = (tc.I * kPairTile + static_cast<int>(rank) * kHalf) / kHalf;
+      const int bz = static_cast<int>(tc.b);
+      const int mat = gd.first_mat + bz;
+      const void* in_map = tmap(a, tc.g, C::kApplyLike ? kTmXfE : kTmAE);
+      // the last step also brings the weight chunk, in the caller's orientation
+      bool w_in = false;
+      bool w_tr = false;
+      if (KIND == kApplyLast) {
+        const MatDesc& md = a.mats[mat];
+        w_in = md.W && last_by_tma(md);
+        w_tr = md.transposed != 0;
+        if (lane == 0 && last_by_tma(md)) {
+          if (md.W) ptx::fence_tmap_acquire(mat_tmap(a, mat, kMtW));
+          if (md.O) ptx::fence_tmap_acquire(mat_tmap(a, mat, kMtO));
+        }
+      }
+      const uint32_t in_bytes = (KIND == kPoly ? kEpiB16 : kEpiF32) + (w_in ? kEpiF32 : 0);
+      auto issue_load = [&](int ch) {
+        // the slot's previous stores must have finished reading it
+        ptx::bulk_wait_read<0>();
+        uint8_t* slot = slots + (ch & 1) * C::kSlot;
+        uint64_t* bar = &eload[ch & 1];
+        const int col0 = tc.J * kPairTile + ch * 32;
+        ptx::mbar_arrive_expect_tx(bar, in_bytes);
+        ptx::tma_load_3d(slot, in_map, bar, col0, row0, bz);
+        if (KIND == kApplyLast && w_in)
+          ptx::tma_load_3d(slot + kOffLastW, mat_tmap(a, mat, kMtW), bar, w_tr ? row0 : col0,
+                           w_tr ? col0 : row0, 0);
+      };
+      if (kInput && lane == 0 && row0 < gd.r) issue_load(0);
+      if (!ptx::mbar_wait(&s.tfull[acc], acc_phase, limit, s.abort_flag)) {
+        raise_abort(a, s);
+        ok = false;
       }
       ptx::tc_fence_after();
-      const GroupDesc& gd = a.groups[tc.g];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lane_base) << 16) + acc * kBN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
+      const int limit_c = C::kApplyLike ? gd.c : gd.r;
 #pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        float v[32];
+      for (int ch = 0; ok && ch < kPairTile / 32; ++ch) {
+        uint8_t* slot = slots + (ch & 1) * C::kSlot;
+        const int col0 = tc.J * kPairTile + ch * 32;
+        // rows or columns past the matrix: nothing to load or store for this chunk
+        const bool live = row0 < gd.r && col0 < limit_c;
+        const bool next_live = row0 < gd.r && col0 + 32 < limit_c && ch + 1 < kPairTile / 32;
+        if (lane == 0) {
+          if (kInput && next_live) issue_load(ch + 1);
+          if (!kInput) ptx::bulk_wait_read<1>();
+        }
         __syncwarp();
+        float v[32];
         ptx::tmem_ld32(taddr + ch * 32, v);
-        if (KIND == kApply) epi_apply(a, gd, tc, trow, ch, v);
-        else epi_symmetric<KIND>(a, gd, tc, trow, ch, v);
+        if (kInput && live) {
+          if (!ptx::mbar_wait(&eload[ch & 1], eload_phase[ch & 1], limit, s.abort_flag)) {
+            raise_abort(a, s);
+            ok = false;
+            break;
+          }
+          eload_phase[ch & 1] ^= 1u;
+        }
+        if (live) {
+          if (KIND == kApply) {
+            epi_apply(a, gd, tc, row0, col0, slot, v, lane);
+          } else if (KIND == kApplyLast) {
+            epi_apply_last(a, gd, tc, row0, col0, slot, v, lane);
+          } else {
+            const int bj = col0 / kHalf;
+            if (bj <= bi) epi_symmetric<KIND>(a, gd, tc, row0, col0, bj < bi, slot, v, lane);
+          }
+        }
+        // one bulk group per chunk (possibly empty), so "all but the newest
+        // group" always means "the chunk that used the other slot"
+        __syncwarp();
+        if (lane == 0) ptx::bulk_commit();
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_tempty[acc]);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) ptx::bulk_wait<0>();
+    if (!ok) {
+      // give an input load still in flight time to land before the pair exits
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (ptx::globaltimer_ns() - t0 < 20000) {
+      }
+    }
+    __syncwarp();
   }
 
   __syncwarp();
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();  // neither CTA leaves while its partner may still use its memory
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, kTmemCols);
+    ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+}
+
+template <int KIND>
+cudaError_t launch_kind(const StageArgs& args, int grid, cudaStream_t stream) {
+  constexpr size_t smem = Cfg<KIND>::kSmem;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(stage_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  stage_tc_kernel<KIND><<<grid, kThreads, smem, stream>>>(args);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t stage_tc_smem_bytes() { return kSmemBytes; }
+size_t stage_tc_smem_bytes() { return Cfg<kGram>::kSmem; }
 
 cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, cudaStream_t stream) {
   if (args.total_tiles <= 0) return cudaSuccess;
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaSuccess;
+  if (grid < 2 || (grid & 1)) return cudaErrorInvalidConfiguration;
   switch (kind) {
-    case kGram:
-      e = cudaFuncSetAttribute(stage_tc_kernel<kGram>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      if (e == cudaSuccess) stage_tc_kernel<kGram><<<grid, kThreads, kSmemBytes, stream>>>(args);
-      break;
-    case kPoly:
-      e = cudaFuncSetAttribute(stage_tc_kernel<kPoly>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      if (e == cudaSuccess) stage_tc_kernel<kPoly><<<grid, kThreads, kSmemBytes, stream>>>(args);
-      break;
+    case kGram: return launch_kind<kGram>(args, grid, stream);
+    case kPoly: return launch_kind<kPoly>(args, grid, stream);
     case kApply:
-      e = cudaFuncSetAttribute(stage_tc_kernel<kApply>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      if (e == cudaSuccess) stage_tc_kernel<kApply><<<grid, kThreads, kSmemBytes, stream>>>(args);
-      break;
-    default:
-      return cudaErrorInvalidValue;
+      return args.last ? launch_kind<kApplyLast>(args, grid, stream) : launch_kind<kApply>(args, grid, stream);
+    default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
 }
 
 }  // namespace muon

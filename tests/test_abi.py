@@ -125,7 +125,8 @@ def expected_workspace(shapes, prec):
     ew = sum(math.ceil(n / 32) * math.ceil(m / 128) for n, m in shapes)
     off = al(ng * 144, 256)          # GroupDesc is 144 bytes
     off = al(off + nm * 80, 256)     # MatDesc is 80 bytes
-    off = al(off + (ng * 6 * 128 if prec == MUON_NS_BF16 else 0), 256)
+    off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
+    off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + ew * 4, 256)
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)

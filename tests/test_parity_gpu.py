@@ -129,3 +129,34 @@ def test_timeout_is_reported_and_the_context_survives():
     # the device still runs the library's kernels
     wl = workloads.make_random([(64, 96)], device="cuda", seed=1)
     assert check_step(wl, "bf16")["O_over_tol"] <= 1.0
+
+
+def test_cuda_graph_replay_matches_eager():
+    """A plan executed from a captured CUDA graph gives the same bits as eager
+    launches (the kernels are deterministic)."""
+    import muon_step_b200 as ms
+    shapes = [(256, 640), (640, 256), (300, 300)]
+    a = workloads.make_random(shapes, device="cuda", seed=17)
+    b = workloads.make_random(shapes, device="cuda", seed=17)
+    h = a.hyper
+    kw = dict(lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"], gamma=h["gamma"])
+    pa = ms.MuonPlan([(a.W[k], a.G[k], a.M[k]) for k in range(a.count)])
+    pb = ms.MuonPlan([(b.W[k], b.G[k], b.M[k]) for k in range(b.count)])
+    wa, wb = pa.alloc_workspace(), pb.alloc_workspace()
+    pa.execute(wa, **kw)
+    pa.execute(wa, **kw)
+    pb.execute(wb, **kw)  # first execute on this workspace copies the descriptors
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        g.capture_begin()
+        pb.execute(wb, stream=s, **kw)
+        g.capture_end()
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for k in range(a.count):
+        assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k])
