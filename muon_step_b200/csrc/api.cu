@@ -115,8 +115,8 @@ struct muon_plan_s {
   int64_t ew_tiles = 0;
   int64_t stage_tiles[kNumKinds] = {0, 0, 0};
   double flops[kNumKinds] = {0, 0, 0};
-  size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_mat_tmaps = 0, off_partial = 0,
-         off_counter = 0, off_scale = 0, desc_bytes = 0, ws_bytes = 0;
+  size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_mat_tmaps = 0, off_tile_mat = 0,
+         off_partial = 0, off_counter = 0, off_scale = 0, desc_bytes = 0, ws_bytes = 0;
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -235,6 +235,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + (tc ? ng * kTmPerGroup * sizeof(CUtensorMap) : 0), 256);
   p->off_mat_tmaps = off;
   off = align_up(off + (tc ? nm * kMtPerMat * sizeof(CUtensorMap) : 0), 256);
+  p->off_tile_mat = off;
+  off = align_up(off + static_cast<size_t>(ew_total) * sizeof(int32_t), 256);
   p->off_partial = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
   p->off_counter = off;
@@ -271,6 +273,10 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   p->blob.assign(p->desc_bytes, 0);
   std::memcpy(p->blob.data() + p->off_groups, p->groups.data(), ng * sizeof(GroupDesc));
   std::memcpy(p->blob.data() + p->off_mats, p->mats.data(), nm * sizeof(MatDesc));
+  auto* tile_mat = reinterpret_cast<int32_t*>(p->blob.data() + p->off_tile_mat);
+  for (size_t k = 0; k < nm; ++k)
+    for (int64_t t = 0; t < p->mats[k].ew_tiles; ++t)
+      tile_mat[p->mats[k].ew_tile_begin + t] = static_cast<int32_t>(k);
   return MUON_OK;
 }
 
@@ -486,6 +492,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   ew.groups = groups;
   ew.mats = mats;
   ew.ws = ws;
+  ew.tile_mat = reinterpret_cast<const int32_t*>(ws + plan->off_tile_mat);
   ew.partial = reinterpret_cast<float*>(ws + plan->off_partial);
   ew.counter = reinterpret_cast<unsigned*>(ws + plan->off_counter);
   ew.scale = scale;

@@ -26,15 +26,6 @@ namespace muon {
 
 namespace {
 
-__device__ __forceinline__ int find_matrix(const MatDesc* mats, int nmats, int64_t tile) {
-  int lo = 0, hi = nmats - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(&mats[mid].ew_tile_begin) <= tile) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -61,7 +52,7 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
 
   const int tid = threadIdx.x;
   const int64_t tile = blockIdx.x;
-  const int mi = find_matrix(a.mats, a.nmats, tile);
+  const int mi = __ldg(&a.tile_mat[tile]);
   const MatDesc md = a.mats[mi];
   const GroupDesc& gd = a.groups[md.group];
   const int64_t n = md.n, m = md.m;
@@ -89,24 +80,35 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
   const bool vec = ((m & 3) == 0) &&
                    (((reinterpret_cast<uintptr_t>(md.G) | reinterpret_cast<uintptr_t>(md.M)) & 15) == 0);
   if (vec) {
-    // thread -> 4 consecutive columns, rows (tid / 32) + 8 k
+    // thread -> 4 consecutive columns, rows (tid / 32) + 8 k; every load is
+    // issued before the first store
+    constexpr int R = kEwRows / 8;
     const int c4 = (tid & 31) * 4;
     const int64_t col = col0 + c4;
+    float4 g4[R], m4[R];
 #pragma unroll
-    for (int k = 0; k < kEwRows / 8; ++k) {
+    for (int k = 0; k < R; ++k) {
+      const int64_t row = row0 + (tid >> 5) + 8 * k;
+      g4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      m4[k] = g4[k];
+      if (row < n && col < m) {  // m % 4 == 0: the 4 columns are all in range
+        const int64_t off = row * m + col;
+        g4[k] = __ldcs(reinterpret_cast<const float4*>(md.G + off));
+        if (a.mode == 0) m4[k] = __ldcs(reinterpret_cast<const float4*>(md.M + off));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
       const int rr = (tid >> 5) + 8 * k;
       const int64_t row = row0 + rr;
       float nv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (row < n && col < m) {  // m % 4 == 0: the 4 columns are all in range
+      if (row < n && col < m) {
         const int64_t off = row * m + col;
-        const float4 g4 = __ldcs(reinterpret_cast<const float4*>(md.G + off));
-        float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (a.mode == 0) m4 = __ldcs(reinterpret_cast<const float4*>(md.M + off));
         float4 mo;
-        nv[0] = step(g4.x, m4.x, &mo.x);
-        nv[1] = step(g4.y, m4.y, &mo.y);
-        nv[2] = step(g4.z, m4.z, &mo.z);
-        nv[3] = step(g4.w, m4.w, &mo.w);
+        nv[0] = step(g4[k].x, m4[k].x, &mo.x);
+        nv[1] = step(g4[k].y, m4[k].y, &mo.y);
+        nv[2] = step(g4[k].z, m4[k].z, &mo.z);
+        nv[3] = step(g4[k].w, m4[k].w, &mo.w);
         if (a.mode == 0) __stcs(reinterpret_cast<float4*>(md.M + off), mo);
         sumsq += nv[0] * nv[0] + nv[1] * nv[1] + nv[2] * nv[2] + nv[3] * nv[3];
         if (!transposed) {
@@ -126,19 +128,31 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
       }
     }
   } else {
-    // scalar path: thread -> one column, rows (tid / 128) + 2 k
+    // scalar path: thread -> one column, rows (tid / 128) + 2 k; loads first
+    constexpr int R = kEwRows / 2;
     const int cc = tid & (kEwCols - 1);
     const int64_t col = col0 + cc;
-    for (int k = 0; k < kEwRows / 2; ++k) {
+    float gs[R], ms[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int64_t row = row0 + (tid >> 7) + 2 * k;
+      gs[k] = 0.f;
+      ms[k] = 0.f;
+      if (row < n && col < m) {
+        const int64_t off = row * m + col;
+        gs[k] = __ldcs(md.G + off);
+        if (a.mode == 0) ms[k] = __ldcs(md.M + off);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
       const int rr = (tid >> 7) + 2 * k;
       const int64_t row = row0 + rr;
       float nv = 0.f;
       if (row < n && col < m) {
         const int64_t off = row * m + col;
-        const float g = __ldcs(md.G + off);
-        const float mp = (a.mode == 0) ? __ldcs(md.M + off) : 0.f;
         float mo;
-        nv = step(g, mp, &mo);
+        nv = step(gs[k], ms[k], &mo);
         if (a.mode == 0) __stcs(md.M + off, mo);
         sumsq += nv * nv;
         if (!transposed) {

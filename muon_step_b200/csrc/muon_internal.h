@@ -105,6 +105,7 @@ struct EwArgs {
   const GroupDesc* groups;
   const MatDesc* mats;
   char* ws;
+  const int32_t* tile_mat;  // matrix of each elementwise tile
   float* partial;         // one partial sum of squares per elementwise tile
   unsigned* counter;      // per-matrix arrival counter (left at zero)
   float* scale;           // per-matrix output 1 / (||N||_F + eps)

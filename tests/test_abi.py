@@ -127,7 +127,8 @@ def expected_workspace(shapes, prec):
     off = al(off + nm * 80, 256)     # MatDesc is 80 bytes
     off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
-    off = al(off + ew * 4, 256)
+    off = al(off + ew * 4, 256)     # matrix of each elementwise tile
+    off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
     off = al(off, 1024)
