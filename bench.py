@@ -162,7 +162,7 @@ class ClockSampler:
 def traffic_from_profile(config):
     """Per-launch DRAM bytes of the Apply kernel from the committed ncu summary
     (null if there is none for this workload)."""
-    path = os.path.join(ROOT, "profiles", f"ns_apply_{config}.md")
+    path = os.path.join(ROOT, "profiles", f"ns_stages_{config}.md")
     if not os.path.exists(path):
         return None
     m = re.search(r"^traffic_per_launch_bytes:\s*([0-9.eE+]+)\s*$", open(path).read(), re.M)

@@ -63,29 +63,35 @@ constexpr int kStageBytes = kABytes + kBBytes;    // 32 KB
 constexpr uint32_t kPairTx = 2 * kStageBytes;     // bytes both CTAs land per ring slot
 constexpr int kPairTile = 256;
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
 constexpr int kEpiF32 = 32 * 32 * 4;              // fp32 32 x 32, 128-byte swizzle
 constexpr int kEpiB16 = 32 * 32 * 2;              // bf16 32 x 32, 64-byte swizzle
-constexpr size_t kBarrierBytes = 256;
+constexpr size_t kBarrierBytes = 512;
 constexpr int kTmapBytes = 128;
 
-// Per-kind layout. Epilogue staging slot (two per warp):
-//   Gram / Poly  [bf16 A in (Poly) | bf16 out | bf16 mirror out]   6 KB
-//   Apply        [fp32 iterate in / out | bf16 iterate out]         6 KB
-//   ApplyLast    [fp32 iterate in / O out | fp32 W in / out]        8 KB
+// Per-kind layout: ring depth and the epilogue staging slot (two per warp,
+// four epilogue warps, one per TMEM lane quarter):
+//   Gram       [bf16 out | bf16 mirror out]                       4 KB
+//   Poly       [bf16 A in | bf16 out | bf16 mirror out]           6 KB
+//   Apply      [fp32 iterate in / out | bf16 iterate out]         6 KB
+//   ApplyLast  [fp32 iterate in / O out | fp32 W in / out]        8 KB
 template <int KIND>
 struct Cfg {
-  static constexpr int kStages = (KIND == kApplyLast) ? 4 : 5;
-  static constexpr int kSlot = (KIND == kApplyLast) ? 2 * kEpiF32 : kEpiF32 + kEpiB16;
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kStages = (KIND == kGram) ? 6 : (KIND == kApplyLast) ? 4 : 5;
+  static constexpr int kSlot = (KIND == kApplyLast) ? 2 * kEpiF32
+                               : (KIND == kGram)    ? 2 * kEpiB16
+                                                    : kEpiF32 + kEpiB16;
   static constexpr int kEpiBytes = kEpiWarps * 2 * kSlot;
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarrierBytes;
   static constexpr bool kApplyLike = (KIND == kApply || KIND == kApplyLast);
   static constexpr int kTiles = kApplyLike ? kApply : KIND;  // which tile tables to walk
+  static constexpr int kChunksPerWarp = (kPairTile / 32) / (kEpiWarps / 4);
+  // symmetric kinds: where the direct and mirrored outputs sit in a slot
+  static constexpr int kOffSymOut = (KIND == kPoly) ? kEpiB16 : 0;
+  static constexpr int kOffSymMirror = kOffSymOut + kEpiB16;
 };
 
-constexpr int kOffSymOut = kEpiB16;
-constexpr int kOffSymMirror = 2 * kEpiB16;
 constexpr int kOffApplyOut16 = kEpiF32;
 constexpr int kOffLastW = kEpiF32;
 
@@ -157,13 +163,13 @@ __device__ __forceinline__ int sw128_f32(int row, int col) { return sw128_chunk(
 
 struct Smem {
   uint8_t* ring;   // stages x (A half | B half)
-  uint8_t* epi;    // kEpiWarps x 2 slots
+  uint8_t* epi;    // epilogue warps x 2 slots
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* drain;
-  uint64_t* eload;  // kEpiWarps x 2
+  uint64_t* eload;  // epilogue warps x 2
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -181,7 +187,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
   s.eload = s.drain + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + 2 * kEpiWarps);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + 2 * Cfg<KIND>::kEpiWarps);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
   return s;
 }
@@ -223,8 +229,8 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const GroupDes
       }
     }
   }
-  uint8_t* st_direct = slot + kOffSymOut;
-  uint8_t* st_mirror = slot + kOffSymMirror;
+  uint8_t* st_direct = slot + Cfg<KIND>::kOffSymOut;
+  uint8_t* st_mirror = slot + Cfg<KIND>::kOffSymMirror;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     Bf16x8 p;
@@ -412,10 +418,11 @@ __device__ __forceinline__ void epi_apply_last(const StageArgs& a, const GroupDe
 // -------------------------------------------------------------- kernel
 
 template <int KIND>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads, 1)
     stage_tc_kernel(const __grid_constant__ StageArgs a) {
   using C = Cfg<KIND>;
   constexpr int kStages = C::kStages;
+  constexpr int kEpiWarps = C::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve<KIND>(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -470,7 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         uint8_t* sa = s.ring + stage * kStageBytes;
         uint8_t* sb = sa + kABytes;
-        if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], kPairTx);
+        const bool diag = !C::kApplyLike && tc.I == tc.J;
+        if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], diag ? kPairTx / 2 : kPairTx);
         const int k0 = kb * kBK;
         if (C::kApplyLike) {
           ptx::tma_load_3d_pair(sa, tmap(a, tc.g, kTmB), leader_full[stage], k0,
@@ -484,7 +492,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const void* tm = (KIND == kGram) ? tmap(a, tc.g, a.xsrc ? kTmXb1K : kTmXb0K)
                                            : tmap(a, tc.g, kTmA);
           ptx::tma_load_3d_pair(sa, tm, leader_full[stage], k0, tc.I * kPairTile + rank * kHalf, bz);
-          ptx::tma_load_3d_pair(sb, tm, leader_full[stage], k0, tc.J * kPairTile + rank * kHalf, bz);
+          // on a diagonal tile each CTA's right-operand half is its left-operand rows
+          if (tc.I != tc.J)
+            ptx::tma_load_3d_pair(sb, tm, leader_full[stage], k0, tc.J * kPairTile + rank * kHalf, bz);
         }
         if (++stage == kStages) {
           stage = 0;
@@ -521,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t sa = ptx::smem_u32(s.ring + stage * kStageBytes);
-        const uint32_t sb = sa + kABytes;
+        const uint32_t sb = (!C::kApplyLike && tc.I == tc.J) ? sa : sa + kABytes;
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t ad = ptx::desc_sw128(sa + k * 32, 16, 1024);
@@ -553,6 +563,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue
     const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may read: 32 * quarter ...
+    const int ch_begin = (ew / 4) * C::kChunksPerWarp;  // this warp's share of the columns
+    const int ch_end = ch_begin + C::kChunksPerWarp;
     uint8_t* slots = s.epi + ew * 2 * C::kSlot;
     uint64_t* eload = s.eload + 2 * ew;
     uint32_t eload_phase[2] = {0u, 0u};
@@ -594,7 +606,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ptx::tma_load_3d(slot + kOffLastW, mat_tmap(a, mat, kMtW), bar, w_tr ? row0 : col0,
                            w_tr ? col0 : row0, 0);
       };
-      if (kInput && lane == 0 && row0 < gd.r) issue_load(0);
+      if (kInput && lane == 0 && row0 < gd.r && tc.J * kPairTile + ch_begin * 32 < (C::kApplyLike ? gd.c : gd.r))
+        issue_load(ch_begin);
       if (!ptx::mbar_wait(&s.tfull[acc], acc_phase, limit, s.abort_flag)) {
         raise_abort(a, s);
         ok = false;
@@ -603,12 +616,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
       const int limit_c = C::kApplyLike ? gd.c : gd.r;
 #pragma unroll 1
-      for (int ch = 0; ok && ch < kPairTile / 32; ++ch) {
+      for (int ch = ch_begin; ok && ch < ch_end; ++ch) {
         uint8_t* slot = slots + (ch & 1) * C::kSlot;
         const int col0 = tc.J * kPairTile + ch * 32;
         // rows or columns past the matrix: nothing to load or store for this chunk
         const bool live = row0 < gd.r && col0 < limit_c;
-        const bool next_live = row0 < gd.r && col0 + 32 < limit_c && ch + 1 < kPairTile / 32;
+        const bool next_live = row0 < gd.r && col0 + 32 < limit_c && ch + 1 < ch_end;
         if (lane == 0) {
           if (kInput && next_live) issue_load(ch + 1);
           if (!kInput) ptx::bulk_wait_read<1>();
@@ -673,7 +686,7 @@ cudaError_t launch_kind(const StageArgs& args, int grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(stage_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  stage_tc_kernel<KIND><<<grid, kThreads, smem, stream>>>(args);
+  stage_tc_kernel<KIND><<<grid, Cfg<KIND>::kThreads, smem, stream>>>(args);
   return cudaGetLastError();
 }
 
