@@ -159,14 +159,32 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+KERNEL_SOURCES = ("muon_step_b200/csrc/ns_tc.cu", "muon_step_b200/csrc/ptx_sm100.cuh",
+                  "muon_step_b200/csrc/stage_common.cuh", "muon_step_b200/csrc/muon_internal.h")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profile(config):
-    """Per-launch DRAM bytes of the Apply kernel from the committed ncu summary
-    (null if there is none for this workload)."""
+    """Per-launch DRAM bytes of the Apply kernel from the committed ncu summary,
+    or None when there is none for this workload or the kernel sources changed
+    since the counters were taken."""
     path = os.path.join(ROOT, "profiles", f"ns_stages_{config}.md")
     if not os.path.exists(path):
         return None
-    m = re.search(r"^traffic_per_launch_bytes:\s*([0-9.eE+]+)\s*$", open(path).read(), re.M)
-    return float(m.group(1)) if m else None
+    text = open(path).read()
+    m = re.search(r"^traffic_per_launch_bytes:\s*([0-9.eE+]+)\s*$", text, re.M)
+    h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)\s*$", text, re.M)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
 
 
 def run_reference(args, rank, world):
