@@ -116,7 +116,10 @@ struct muon_plan_s {
   int64_t stage_tiles[kNumKinds] = {0, 0, 0};
   double flops[kNumKinds] = {0, 0, 0};
   size_t off_groups = 0, off_mats = 0, off_tmaps = 0, off_mat_tmaps = 0, off_tile_mat = 0,
-         off_partial = 0, off_counter = 0, off_scale = 0, desc_bytes = 0, ws_bytes = 0;
+         off_small = 0, off_partial = 0, off_counter = 0, off_scale = 0, desc_bytes = 0,
+         ws_bytes = 0;
+  std::vector<int32_t> small_mats;  // internal indices run by the small-matrix kernel
+  std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -176,7 +179,13 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     gd.count = static_cast<int32_t>(members[g].size());
     gd.first_mat = static_cast<int32_t>(p->mats.size());
     double fl[kNumKinds] = {0, 0, 0};
-    if (tc) {
+    gd.small = (tc && r <= kSmallMax && c <= kSmallMax) ? 1 : 0;
+    if (gd.small) {
+      // one CTA per matrix, dense 128 x 128 products; count the useful FLOPs
+      fl[kGram] = 2.0 * r * r * static_cast<double>(c);
+      fl[kPoly] = 2.0 * r * r * static_cast<double>(r);
+      for (int k = 0; k < kNumKinds; ++k) gd.tiles_per_mat[k] = 0;
+    } else if (tc) {
       // pair tiles of 256 x 256; the symmetric stages run those on or below
       // the diagonal and keep the 128 x 128 blocks on or below it
       const int64_t rb = cdiv(r, 128);
@@ -216,6 +225,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
       md.flags = 0;
       if (md.W && rows16 && (reinterpret_cast<uintptr_t>(md.W) & 15) == 0) md.flags |= kMatWTma;
       if (md.O && rows16 && (reinterpret_cast<uintptr_t>(md.O) & 15) == 0) md.flags |= kMatOTma;
+      if (gd.small) p->small_mats.push_back(static_cast<int32_t>(p->mats.size()));
       md.ew_tile_begin = ew_total;
       md.ew_tiles = cdiv(md.n, kEwRows) * cdiv(md.m, kEwCols);
       ew_total += md.ew_tiles;
@@ -237,6 +247,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + (tc ? nm * kMtPerMat * sizeof(CUtensorMap) : 0), 256);
   p->off_tile_mat = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(int32_t), 256);
+  p->off_small = off;
+  off = align_up(off + p->small_mats.size() * sizeof(int32_t), 256);
   p->off_partial = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
   p->off_counter = off;
@@ -273,6 +285,18 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   p->blob.assign(p->desc_bytes, 0);
   std::memcpy(p->blob.data() + p->off_groups, p->groups.data(), ng * sizeof(GroupDesc));
   std::memcpy(p->blob.data() + p->off_mats, p->mats.data(), nm * sizeof(MatDesc));
+  if (!p->small_mats.empty())
+    std::memcpy(p->blob.data() + p->off_small, p->small_mats.data(), p->small_mats.size() * sizeof(int32_t));
+  // the launch list of one execute
+  p->launch_kinds.assign(1, 0);
+  if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
+  if (p->stage_tiles[kApply] > 0) {
+    for (int k = 0; k < p->steps; ++k) {
+      p->launch_kinds.push_back(1);
+      p->launch_kinds.push_back(2);
+      p->launch_kinds.push_back(k + 1 == p->steps ? 4 : 3);
+    }
+  }
   auto* tile_mat = reinterpret_cast<int32_t*>(p->blob.data() + p->off_tile_mat);
   for (size_t k = 0; k < nm; ++k)
     for (int64_t t = 0; t < p->mats[k].ew_tiles; ++t)
@@ -346,7 +370,7 @@ muon_status_t record(muon_plan_s* p, int slot, cudaStream_t stream) {
   return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
-int launch_count(const muon_plan_s* p) { return 1 + 3 * p->steps; }
+int launch_count(const muon_plan_s* p) { return static_cast<int>(p->launch_kinds.size()); }
 
 }  // namespace
 
@@ -427,16 +451,8 @@ muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int m
   if (!plan || !count) return MUON_ERR_INVALID_ARG;
   const int n = launch_count(plan);
   *count = n;
-  if (kinds) {
-    for (int k = 0; k < n && k < max_kinds; ++k) {
-      if (k == 0) kinds[k] = 0;
-      else {
-        const int kind = (k - 1) % 3;
-        const bool last = (k - 1) / 3 == plan->steps - 1;
-        kinds[k] = (kind == kApply) ? (last ? 4 : 3) : kind + 1;
-      }
-    }
-  }
+  if (kinds)
+    for (int k = 0; k < n && k < max_kinds; ++k) kinds[k] = plan->launch_kinds[k];
   return MUON_OK;
 }
 
@@ -511,6 +527,30 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   const bool tc = plan->prec == MUON_NS_BF16;
   const int sms = g_num_sms[dev];
   int slot = 2;
+  if (!plan->small_mats.empty()) {
+    SmallArgs sm{};
+    sm.groups = groups;
+    sm.mats = mats;
+    sm.tmaps = ws + plan->off_tmaps;
+    sm.ws = ws;
+    sm.scale = scale;
+    sm.small_mats = reinterpret_cast<const int32_t*>(ws + plan->off_small);
+    sm.err = err;
+    sm.nsmall = static_cast<int64_t>(plan->small_mats.size());
+    sm.steps = plan->steps;
+    if (plan->mode == 0) {
+      sm.lr = hyper->lr;
+      sm.wd = hyper->weight_decay;
+      sm.gamma = hyper->gamma;
+    }
+    sm.wait_limit_ns = limit;
+    for (int k = 0; k < 3 * plan->steps; ++k) sm.abc[k] = plan->abc[k];
+    const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (launch_small(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+  }
+  if (plan->stage_tiles[kApply] == 0) return MUON_OK;
   for (int k = 0; k < plan->steps; ++k) {
     for (int kind = 0; kind < kNumKinds; ++kind) {
       StageArgs sa{};

@@ -17,6 +17,10 @@ cudaError_t launch_elementwise(const EwArgs& args, cudaStream_t stream);
 cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid,
                             cudaStream_t stream);
 
+// Every Newton-Schulz step and the update for the small matrices, one CTA
+// per matrix (bf16 precision).
+cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream);
+
 // The same stage in fp32 on the CUDA cores (validation precision).
 cudaError_t launch_stage_simt(StageKind kind, const StageArgs& args, int grid,
                               cudaStream_t stream);

@@ -21,6 +21,10 @@ constexpr int kPairM = 256;
 constexpr int kPairN = 256;
 constexpr int kBK = 64;
 
+// Matrices with min(n, m) <= kSmallMax and max(n, m) <= kSmallMax run the
+// whole Newton-Schulz iteration in one CTA (bf16 precision).
+constexpr int kSmallMax = 128;
+
 // fp32 validation tile shape.
 constexpr int kSBM = 64;
 constexpr int kSBN = 64;
@@ -59,6 +63,8 @@ struct GroupDesc {
   int32_t ldc, ldr;      // leading dimensions (elements) of r x c and r x r buffers
   int32_t count;         // matrices in this group
   int32_t first_mat;     // internal index of the group's first matrix
+  int32_t small;         // 1: runs in the small-matrix kernel, no stage tiles
+  int32_t pad0;
   int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate (fp32 mode ping-pongs)
   int64_t xb_off[2];     // bf16 iterate, ping-pong
   int64_t a_off, b_off;  // A = X X^T and B = bA + cA^2 (bf16, or fp32 in fp32 mode)
@@ -116,6 +122,22 @@ struct EwArgs {
   int32_t nesterov;
   int32_t write_bf16;     // bf16 mode writes the bf16 operand copy too
   float mu, eps;
+};
+
+// Small-matrix kernel arguments (one CTA per matrix, every step on chip).
+struct SmallArgs {
+  const GroupDesc* groups;
+  const MatDesc* mats;
+  const void* tmaps;      // group tensor maps (the bf16 iterate, K-major box)
+  char* ws;
+  const float* scale;
+  const int32_t* small_mats;  // internal indices of the small matrices
+  int* err;
+  int64_t nsmall;
+  int32_t steps;
+  float lr, wd, gamma;    // update hyper-parameters
+  uint64_t wait_limit_ns;
+  float abc[kMaxSteps * 3];
 };
 
 // error bits in the device error word

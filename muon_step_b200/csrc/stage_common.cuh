@@ -41,11 +41,15 @@ struct UpdateConsts {
   float step;  // lr gamma sqrt(max(n, m))
 };
 
-__device__ __forceinline__ UpdateConsts update_consts(const StageArgs& a, int c) {
+__device__ __forceinline__ UpdateConsts update_consts_raw(float lr, float wd, float gamma, int c) {
   UpdateConsts u;
-  u.keep = 1.0f - a.lr * a.wd;
-  u.step = a.lr * a.gamma * sqrtf(static_cast<float>(c));
+  u.keep = 1.0f - lr * wd;
+  u.step = lr * gamma * sqrtf(static_cast<float>(c));
   return u;
+}
+
+__device__ __forceinline__ UpdateConsts update_consts(const StageArgs& a, int c) {
+  return update_consts_raw(a.lr, a.wd, a.gamma, c);
 }
 
 __device__ __forceinline__ void write_update(const MatDesc& md, const UpdateConsts& u,

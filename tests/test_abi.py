@@ -117,22 +117,27 @@ def expected_workspace(shapes, prec):
     """Independent restatement of the documented layout: per shape group an
     fp32 iterate (two in fp32 mode), two bf16 iterates (bf16 mode), A and B;
     rows padded to multiples of 8 elements; regions 1024-byte aligned."""
-    groups = {}
+    groups, order = {}, []
     for n, m in shapes:
-        groups.setdefault((min(n, m), max(n, m)), []).append((n, m))
+        key = (min(n, m), max(n, m))
+        if key not in groups:
+            order.append(key)
+        groups.setdefault(key, []).append((n, m))
     al = lambda x, a: (x + a - 1) // a * a
     ng, nm = len(groups), len(shapes)
     ew = sum(math.ceil(n / 32) * math.ceil(m / 128) for n, m in shapes)
-    off = al(ng * 144, 256)          # GroupDesc is 144 bytes
+    off = al(ng * 152, 256)          # GroupDesc is 152 bytes
     off = al(off + nm * 80, 256)     # MatDesc is 80 bytes
     off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + ew * 4, 256)     # matrix of each elementwise tile
+    small = [(n, m) for n, m in shapes if prec == MUON_NS_BF16 and max(n, m) <= 128]
+    off = al(off + len(small) * 4, 256)  # small-matrix list
     off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
     off = al(off, 1024)
-    for (r, c), mem in groups.items():
+    for (r, c), mem in sorted(groups.items(), key=lambda kv: order.index(kv[0])):
         k = len(mem)
         x = k * r * al(c, 8)
         a = k * r * al(r, 8)
@@ -160,14 +165,26 @@ def test_workspace_size_matches_layout(lib, prec):
     assert m.value == n.value
 
 
-def test_launch_list(lib):
-    st, plan = create(lib, [(64, 64)])
+def launch_list(lib, shapes, prec=MUON_NS_BF16):
+    st, plan = create(lib, shapes, prec)
+    assert st == MUON_OK
     cnt = ctypes.c_int()
-    kinds = (ctypes.c_int * 64)()
-    assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 64) == MUON_OK
+    kinds = (ctypes.c_int * 128)()
+    assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 128) == MUON_OK
     lib.muon_plan_destroy(plan)
-    assert cnt.value == 31
-    assert list(kinds[:31]) == [0] + [1, 2, 3] * 9 + [1, 2, 4]
+    return list(kinds[:cnt.value])
+
+
+def test_launch_list(lib):
+    grouped = [1, 2, 3] * 9 + [1, 2, 4]
+    # matrices up to 128 x 128 run in the one-CTA small-matrix kernel (kind 5)
+    assert launch_list(lib, [(64, 64)]) == [0, 5]
+    assert launch_list(lib, [(128, 128), (1, 1), (7, 100)]) == [0, 5]
+    assert launch_list(lib, [(300, 400)]) == [0] + grouped
+    assert launch_list(lib, [(129, 64)]) == [0] + grouped
+    assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 5] + grouped
+    # the fp32 validation precision has no small-matrix kernel
+    assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + grouped
 
 
 def test_flops_count_the_computed_tiles(lib):
@@ -197,7 +214,7 @@ def test_ns_plan_arguments(lib):
 
 
 def test_timing_events_need_two_per_launch(lib):
-    st, plan = create(lib, [(8, 8)])
+    st, plan = create(lib, [(300, 300)])
     ev = (ctypes.c_void_p * 62)(*([FAKE] * 62))
     assert lib.muon_plan_set_events(plan, ev, 61) == MUON_ERR_INVALID_ARG
     assert lib.muon_plan_set_events(plan, ev, 62) == MUON_OK
