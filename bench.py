@@ -72,6 +72,22 @@ def apply_bytes(shapes):
     return sum(2.0 * min(n, m) ** 2 + 12.0 * min(n, m) * max(n, m) for n, m in shapes)
 
 
+def max_over_ranks(x, device, world):
+    """The job-wide maximum of a per-rank number (the slowest rank's time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank, world, steps, ms_max):
+    """Whole-job throughput: the FLOPs of every rank over the slowest rank's time."""
+    return flops_per_rank * world * steps / (ms_max / 1e3) / 1e12
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -328,13 +344,10 @@ def main():
     if status != 0:
         raise SystemExit(f"device error status {status}")
 
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms_total, dev, world)
     ms_per_step = ms_max / args.steps
     flops_rank = metric_flops(wl.shapes, ns_steps)
-    value = flops_rank * world * args.steps / (ms_max / 1e3) / 1e12
+    value = job_tflops(flops_rank, world, args.steps, ms_max)
 
     # per-kernel durations over the timed region
     per_kind = {}
@@ -407,12 +420,10 @@ def main():
         e_e.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([e_s.elapsed_time(e_e)], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": flops_rank * world * args.steps / (float(te.item()) / 1e3) / 1e12,
+        te = max_over_ranks(e_s.elapsed_time(e_e), dev, world)
+        e2e = {"value": job_tflops(flops_rank, world, args.steps, te),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": float(te.item()) / args.steps}
+               "ms_per_step": te / args.steps}
         assert ms.sync_status() == 0
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)

@@ -160,3 +160,36 @@ def test_cuda_graph_replay_matches_eager():
     assert ms.sync_status() == 0
     for k in range(a.count):
         assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k])
+
+
+def test_distributed_step_world_one_matches_plan():
+    """DistributedMuon with its default compute (the library's plan over the
+    owned matrices) and an NCCL group of one rank equals a direct plan."""
+    import datetime
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    import muon_step_b200 as ms
+    from muon_step_b200.distributed import DistributedMuon
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        shapes = [(300, 500), (500, 300), (64, 64)]
+        a = workloads.make_random(shapes, device="cuda", seed=23)
+        b = workloads.make_random(shapes, device="cuda", seed=23)
+        opt = DistributedMuon([(a.W[k], a.G[k], a.M[k]) for k in range(a.count)])
+        opt.step()
+        plan = ms.MuonPlan([(b.W[k], b.G[k], b.M[k]) for k in range(b.count)])
+        plan.execute()
+        torch.cuda.synchronize()
+        for k in range(a.count):
+            assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k])
+    finally:
+        dist.destroy_process_group()
