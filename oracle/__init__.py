@@ -15,4 +15,7 @@ from .muon_oracle import (  # noqa: F401
     ns_step,
     orient,
     rescale,
+    rescale_none,
+    rescale_unit_rms,
+    SCALE_MODES,
 )

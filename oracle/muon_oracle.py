@@ -120,6 +120,27 @@ def rescale(O_prime: np.ndarray, n: int, m: int, gamma: float) -> np.ndarray:
     return O_prime * (np.sqrt(float(max(n, m))) * gamma)
 
 
+def rescale_unit_rms(O_prime: np.ndarray, gamma: float) -> np.ndarray:
+    """O = gamma * O' / RMS(O'): the update normalised to unit RMS, then scaled.
+
+    [V4-breakdown] section "分布式工程", the Megatron-Bridge recipe's
+    muon_scale_mode "unit_rms_norm" with muon_extra_scale_factor gamma
+    ("把更新显式归一到单位 RMS 再乘 0.2"). A zero O' stays zero.
+    """
+    rms = np.sqrt(np.mean(O_prime * O_prime))
+    return O_prime * (gamma / rms) if rms > 0.0 else np.zeros_like(O_prime)
+
+
+def rescale_none(O_prime: np.ndarray, gamma: float) -> np.ndarray:
+    """O = gamma * O': no shape-dependent rescale, as in the original Muon
+    ([V4-breakdown] Algorithm 1 discussion: the original Muon had neither
+    weight decay nor the RMS rescale; gamma = 1 reproduces it)."""
+    return O_prime * gamma
+
+
+SCALE_MODES = ("shape", "unit_rms", "none")
+
+
 def decay_and_update(W: np.ndarray, O: np.ndarray, lr: float, wd: float) -> np.ndarray:
     """Decoupled weight decay and step: W_t = W_{t-1} (1 - lr*wd) - lr * O_t.
 
@@ -138,13 +159,15 @@ def ns_orthogonalize(X: np.ndarray, schedule=HYBRID_SCHEDULE,
 
 
 def muon_step(W, G, M_prev, lr=0.02, mu=0.95, wd=0.1, gamma=0.2,
-              nesterov_on=True, schedule=HYBRID_SCHEDULE, eps=DEFAULT_EPS):
+              nesterov_on=True, schedule=HYBRID_SCHEDULE, eps=DEFAULT_EPS, scale_mode="shape"):
     """One Muon step for one n x m matrix, all in float64.
 
     Returns (W_t, M_t, O'_t) where O'_t is the orthogonalised direction before
     the RMS rescale, in W's orientation. Follows [V4-breakdown] Algorithm 1 and
     [V4-book] §5 Algorithm 1 step by step. With ``nesterov_on`` false the
-    orthogonaliser's input is M_t itself (the original Muon).
+    orthogonaliser's input is M_t itself (the original Muon). ``scale_mode``
+    picks the update's scale: "shape" (sqrt(max(n, m)) gamma, the default),
+    "unit_rms" (gamma / RMS(O')) or "none" (gamma).
     """
     W = np.asarray(W, dtype=np.float64)
     G = np.asarray(G, dtype=np.float64)
@@ -153,6 +176,13 @@ def muon_step(W, G, M_prev, lr=0.02, mu=0.95, wd=0.1, gamma=0.2,
     M = momentum(M_prev, G, mu)
     N = nesterov(M, G, mu) if nesterov_on else M
     O_prime = ns_orthogonalize(N, schedule, eps)
-    O = rescale(O_prime, n, m, gamma)
+    if scale_mode == "shape":
+        O = rescale(O_prime, n, m, gamma)
+    elif scale_mode == "unit_rms":
+        O = rescale_unit_rms(O_prime, gamma)
+    elif scale_mode == "none":
+        O = rescale_none(O_prime, gamma)
+    else:
+        raise ValueError(scale_mode)
     W_new = decay_and_update(W, O, lr, wd)
     return W_new, M, O_prime

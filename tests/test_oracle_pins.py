@@ -372,3 +372,35 @@ def test_planted_schedule_mistakes_are_caught(golden_dir, monkeypatch):
                             _f(X, schedule, eps))
         assert _pins(golden_dir), "schedule mistake passed every pin"
         monkeypatch.undo()
+
+
+# ----------------------------------------------------------------------------
+# scale modes
+# ----------------------------------------------------------------------------
+
+def test_unit_rms_mode_has_rms_gamma_and_matches_shape_mode():
+    """unit_rms_norm: RMS(O) = gamma exactly; in theory equal to the shape
+    rescale because RMS(O') ~ sqrt(1 / max(n, m)) ("Muon 优化器完全拆解…",
+    section "分布式工程": "两者在理论上等价"), so on well-conditioned inputs
+    the two agree within the band."""
+    rng = np.random.default_rng(31)
+    for n, m in [(48, 48), (32, 96), (96, 32)]:
+        N = matrix_with_spectrum(rng, n, m, rng.uniform(0.7, 1.2, min(n, m)))
+        Z = np.zeros((n, m))
+        W_u, _, O_p = oracle.muon_step(Z, N, Z, lr=1.0, mu=0.0, wd=0.0, gamma=0.2, scale_mode="unit_rms")
+        assert abs(np.sqrt(np.mean(W_u ** 2)) - 0.2) < 1e-12
+        W_s, _, _ = oracle.muon_step(Z, N, Z, lr=1.0, mu=0.0, wd=0.0, gamma=0.2, scale_mode="shape")
+        assert rel(W_u, W_s) <= 2.1e-3
+
+
+def test_none_mode_is_the_plain_direction_and_zero_stays_zero():
+    rng = np.random.default_rng(32)
+    W = rng.standard_normal((20, 30))
+    G = rng.standard_normal((20, 30))
+    W_n, _, O_p = oracle.muon_step(W, G, np.zeros_like(W), lr=0.1, mu=0.9, wd=0.01, gamma=1.0,
+                                   scale_mode="none")
+    assert np.allclose(W_n, W * (1 - 0.1 * 0.01) - 0.1 * O_p, rtol=1e-14, atol=1e-15)
+    Z = np.zeros_like(W)
+    for mode in ("unit_rms", "none"):
+        W_z, _, _ = oracle.muon_step(W, Z, Z, lr=0.1, wd=0.01, scale_mode=mode)
+        assert np.array_equal(W_z, W * (1 - 0.1 * 0.01))
