@@ -104,6 +104,13 @@ typedef struct {
   int nesterov;
 } muon_hyper_t;
 
+/* How O' is scaled into the update O (W <- W (1 - lr wd) - lr O):
+ *   SHAPE     O = O' sqrt(max(n, m)) gamma   ([V4-breakdown] Algorithm 1; default)
+ *   UNIT_RMS  O = O' gamma / RMS(O')         ([V4-breakdown] "分布式工程": the
+ *             Megatron-Bridge recipe's unit_rms_norm scale mode; O' = 0 gives O = 0)
+ *   NONE      O = O' gamma                   (the original Muon with gamma = 1) */
+typedef enum { MUON_SCALE_SHAPE = 0, MUON_SCALE_UNIT_RMS = 1, MUON_SCALE_NONE = 2 } muon_scale_mode_t;
+
 typedef struct muon_plan_s* muon_plan_t;
 
 /* ---------------------------------------------------------------- plans
@@ -125,6 +132,11 @@ MUON_API muon_status_t muon_plan_create_ns(const muon_ns_matrix_t* mats, int cou
                                   muon_precision_t prec, const muon_ns_schedule_t* sched,
                                   muon_plan_t* plan);
 
+/* Select the update scale of later executes (default MUON_SCALE_SHAPE). In
+ * UNIT_RMS mode the last step adds a per-matrix reduction and an elementwise
+ * update pass for matrices larger than 128 x 128. */
+MUON_API muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode);
+
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */
 MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes);
 
@@ -135,7 +147,9 @@ MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* h
                                 size_t workspace_bytes, void* stream);
 
 /* Number of kernel launches one execute issues, and the kind of each
- * (0 momentum/norm/cast, 1 Gram, 2 polynomial, 3 apply, 4 apply + update). */
+ * (0 momentum/norm/cast, 1 Gram, 2 polynomial, 3 apply, 4 apply + update,
+ * 5 small-matrix kernel (all steps and the update of matrices up to
+ * 128 x 128), 6 per-matrix RMS reduction, 7 update pass). */
 MUON_API muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds);
 
 /* Optional timing: `events` holds 2 * launches cudaEvent_t (as void*); each

@@ -148,7 +148,8 @@ class _PlanBase:
 class MuonPlan(_PlanBase):
     """A planned Muon step over a fixed list of (W, G, M[, O]) fp32 CUDA matrices."""
 
-    def __init__(self, params: Iterable, precision="bf16", schedule=None, eps=None):
+    def __init__(self, params: Iterable, precision="bf16", schedule=None, eps=None,
+                 scale_mode="shape"):
         items = []
         self._tensors = []
         for k, p in enumerate(params):
@@ -172,6 +173,17 @@ class MuonPlan(_PlanBase):
                                             ctypes.byref(sched) if sched else None,
                                             ctypes.byref(plan)), "muon_plan_create")
         self._plan = plan
+        if scale_mode != "shape":
+            self.set_scale_mode(scale_mode)
+
+    SCALE_MODES = {"shape": 0, "unit_rms": 1, "none": 2}
+
+    def set_scale_mode(self, mode):
+        """Update scale: "shape" (O' sqrt(max(n, m)) gamma, default), "unit_rms"
+        (O' gamma / RMS(O')) or "none" (O' gamma). Timing events must be set
+        again afterwards (the launch list may change)."""
+        _check(_lib.load().muon_plan_set_scale_mode(self._plan, self.SCALE_MODES[mode]),
+               "muon_plan_set_scale_mode")
 
     def execute(self, workspace=None, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2,
                 nesterov=True, stream=None):

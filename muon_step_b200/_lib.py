@@ -20,13 +20,17 @@ MUON_NS_FP32 = 1
 
 MUON_STATIC_SCRATCH_BYTES = 64 << 20
 
+MUON_SCALE_SHAPE = 0
+MUON_SCALE_UNIT_RMS = 1
+MUON_SCALE_NONE = 2
+
 # every symbol include/muon_step.h declares
 EXPORTS = (
     "muon_plan_create", "muon_plan_create_ns", "muon_plan_workspace_size", "muon_plan_execute",
     "muon_plan_launches", "muon_plan_set_events", "muon_plan_flops", "muon_plan_destroy",
     "muon_workspace_size", "muon_step", "ns_workspace_size", "ns_orthogonalize",
     "muon_sync_status", "muon_status_string", "muon_abi_version", "muon_set_wait_limit_ns",
-    "muon_wait_probe", "muon_step_static_scratch",
+    "muon_wait_probe", "muon_step_static_scratch", "muon_plan_set_scale_mode",
 )
 
 
@@ -75,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_plan_set_events": (st, [vp, P(vp), ctypes.c_int]),
         "muon_plan_flops": (st, [vp, P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_double)]),
         "muon_plan_destroy": (None, [vp]),
+        "muon_plan_set_scale_mode": (st, [vp, ctypes.c_int]),
         "muon_workspace_size": (st, [P(MuonParam), ctypes.c_int, ctypes.c_int, P(ctypes.c_size_t)]),
         "muon_step": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                            ctypes.c_float, ctypes.c_int, P(MuonNsSchedule), ctypes.c_int, vp,

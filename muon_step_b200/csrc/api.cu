@@ -119,7 +119,11 @@ struct muon_plan_s {
          off_small = 0, off_partial = 0, off_counter = 0, off_scale = 0, desc_bytes = 0,
          ws_bytes = 0;
   std::vector<int32_t> small_mats;  // internal indices run by the small-matrix kernel
-  std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small
+  std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small,
+                                    // 6 RMS reduction, 7 update pass (unit-RMS scale)
+  int scale_mode = MUON_SCALE_SHAPE;
+  int sumsq_per_tile = 1;           // sum-of-squares slots per Apply tile (unit-RMS scale)
+  size_t off_sumsq = 0, off_factor = 0;
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -144,6 +148,24 @@ muon_status_t set_schedule(muon_plan_s* p, const muon_ns_schedule_t* s) {
   p->abc.assign(s->abc, s->abc + 3 * s->steps);
   p->eps = s->eps;
   return MUON_OK;
+}
+
+// The launch list of one execute (depends on the scale mode).
+void make_launch_list(muon_plan_s* p) {
+  const bool unit = p->scale_mode == MUON_SCALE_UNIT_RMS;
+  p->launch_kinds.assign(1, 0);
+  if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
+  if (p->stage_tiles[kApply] > 0) {
+    for (int k = 0; k < p->steps; ++k) {
+      p->launch_kinds.push_back(1);
+      p->launch_kinds.push_back(2);
+      p->launch_kinds.push_back(k + 1 == p->steps && !unit ? 4 : 3);
+    }
+    if (unit) {
+      p->launch_kinds.push_back(6);
+      p->launch_kinds.push_back(7);
+    }
+  }
 }
 
 // Build groups, tiles, flop counts and the workspace layout from `mats`
@@ -255,6 +277,12 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + nm * sizeof(unsigned), 256);
   p->off_scale = off;
   off = align_up(off + nm * sizeof(float), 256);
+  // unit-RMS scale: sums of squares of O' per Apply tile, then gamma / RMS per matrix
+  p->sumsq_per_tile = tc ? 8 : 1;  // tensor cores: 2 CTAs x 4 epilogue warps per tile
+  p->off_sumsq = off;
+  off = align_up(off + static_cast<size_t>(p->stage_tiles[kApply]) * p->sumsq_per_tile * sizeof(float), 256);
+  p->off_factor = off;
+  off = align_up(off + nm * sizeof(float), 256);
   p->desc_bytes = off;
   off = align_up(off, 1024);
   for (auto& gd : p->groups) {
@@ -287,16 +315,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   std::memcpy(p->blob.data() + p->off_mats, p->mats.data(), nm * sizeof(MatDesc));
   if (!p->small_mats.empty())
     std::memcpy(p->blob.data() + p->off_small, p->small_mats.data(), p->small_mats.size() * sizeof(int32_t));
-  // the launch list of one execute
-  p->launch_kinds.assign(1, 0);
-  if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
-  if (p->stage_tiles[kApply] > 0) {
-    for (int k = 0; k < p->steps; ++k) {
-      p->launch_kinds.push_back(1);
-      p->launch_kinds.push_back(2);
-      p->launch_kinds.push_back(k + 1 == p->steps ? 4 : 3);
-    }
-  }
+  make_launch_list(p);
   auto* tile_mat = reinterpret_cast<int32_t*>(p->blob.data() + p->off_tile_mat);
   for (size_t k = 0; k < nm; ++k)
     for (int64_t t = 0; t < p->mats[k].ew_tiles; ++t)
@@ -543,6 +562,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       sm.wd = hyper->weight_decay;
       sm.gamma = hyper->gamma;
     }
+    sm.scale_mode = plan->scale_mode;
     sm.wait_limit_ns = limit;
     for (int k = 0; k < 3 * plan->steps; ++k) sm.abc[k] = plan->abc[k];
     const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
@@ -551,6 +571,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
     if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
   }
   if (plan->stage_tiles[kApply] == 0) return MUON_OK;
+  const bool unit = plan->scale_mode == MUON_SCALE_UNIT_RMS;
   for (int k = 0; k < plan->steps; ++k) {
     for (int kind = 0; kind < kNumKinds; ++kind) {
       StageArgs sa{};
@@ -563,8 +584,16 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       sa.err = err;
       sa.total_tiles = plan->stage_tiles[kind];
       sa.ngroups = static_cast<int32_t>(plan->groups.size());
+      const bool last = k == plan->steps - 1;
       sa.first = k == 0;
-      sa.last = k == plan->steps - 1;
+      // unit-RMS scale: the last Apply keeps O' and its sums of squares; the
+      // update comes after the per-matrix reduction
+      sa.last = last && !unit;
+      sa.scale_mode = plan->scale_mode;
+      if (unit && last && kind == kApply) {
+        sa.sumsq_per_tile = plan->sumsq_per_tile;
+        sa.sumsq = reinterpret_cast<float*>(ws + plan->off_sumsq);
+      }
       sa.xsrc = k & 1;
       sa.a = plan->abc[3 * k];
       sa.b = plan->abc[3 * k + 1];
@@ -589,6 +618,40 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
     }
   }
+  if (unit) {
+    FinishArgs fa{};
+    fa.groups = groups;
+    fa.mats = mats;
+    fa.tile_mat = reinterpret_cast<const int32_t*>(ws + plan->off_tile_mat);
+    fa.ws = ws;
+    fa.sumsq = reinterpret_cast<const float*>(ws + plan->off_sumsq);
+    fa.factor = reinterpret_cast<float*>(ws + plan->off_factor);
+    fa.total_tiles = plan->ew_tiles;
+    fa.nmats = static_cast<int32_t>(plan->mats.size());
+    // fp32 path: the last step wrote buffer (steps & 1); tensor cores update in place
+    fa.xf_slot = tc ? 0 : (plan->steps & 1);
+    fa.sumsq_per_tile = plan->sumsq_per_tile;
+    fa.apply_kind = kApply;
+    fa.lr = hyper->lr;
+    fa.wd = hyper->weight_decay;
+    fa.gamma = hyper->gamma;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (launch_rms_reduce(fa, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (launch_finish(fa, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+  }
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode) {
+  if (!plan || plan->mode != 0) return MUON_ERR_INVALID_ARG;
+  if (mode != MUON_SCALE_SHAPE && mode != MUON_SCALE_UNIT_RMS && mode != MUON_SCALE_NONE)
+    return MUON_ERR_INVALID_ARG;
+  plan->scale_mode = mode;
+  make_launch_list(plan);
+  plan->events.clear();  // the launch list may have changed: timing must be set again
   return MUON_OK;
 }
 

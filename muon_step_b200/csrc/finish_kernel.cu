@@ -1,0 +1,117 @@
+// Update pass of the unit-RMS scale mode for matrices on the grouped (or
+// fp32) path.
+//
+// "Muon 优化器完全拆解…", section "分布式工程": the Megatron-Bridge recipe scales
+// the update to unit RMS and then by an extra factor, O = gamma O' / RMS(O').
+// RMS(O') needs all of O' before any element of W can move, so here the last
+// Apply stage keeps O' in the fp32 iterate and records sums of squares per
+// tile; then
+//
+//   rms_reduce_kernel   one CTA per matrix adds its tiles' sums in a fixed
+//                       order (double) and stores gamma / RMS(O') (0 when
+//                       O' = 0);
+//   finish_kernel       W <- W (1 - lr wd) - lr factor O' (and O = O'), over
+//                       32 x 128 tiles of the caller's matrix; when the
+//                       iterate is the transpose, the tile is read through
+//                       shared memory so every global access stays coalesced.
+//
+// HBM-bound: 4 B of O' read, 8 B of W read and written per element.
+#include "kernels.cuh"
+#include "stage_common.cuh"
+
+namespace muon {
+
+namespace {
+
+__global__ void __launch_bounds__(256) rms_reduce_kernel(const __grid_constant__ FinishArgs a) {
+  __shared__ double part[8];
+  const int mat = blockIdx.x;
+  const MatDesc& md = a.mats[mat];
+  const GroupDesc& gd = a.groups[md.group];
+  if (gd.small) return;  // the small-matrix kernel has already updated it
+  const int64_t per = gd.tiles_per_mat[a.apply_kind];
+  const int64_t first = (gd.tile_base[a.apply_kind] + md.index * per) * a.sumsq_per_tile;
+  const int64_t count = per * a.sumsq_per_tile;
+  double acc = 0.0;
+  for (int64_t k = threadIdx.x; k < count; k += blockDim.x) acc += static_cast<double>(a.sumsq[first + k]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < 8; ++w) tot += part[w];
+    const double rms = sqrt(tot / (static_cast<double>(md.n) * static_cast<double>(md.m)));
+    a.factor[mat] = rms > 0.0 ? static_cast<float>(static_cast<double>(a.gamma) / rms) : 0.f;
+  }
+}
+
+__global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ FinishArgs a) {
+  __shared__ float stage[kEwRows][kEwCols + 1];
+  const int tid = threadIdx.x;
+  const int64_t tile = blockIdx.x;
+  const int mat = __ldg(&a.tile_mat[tile]);
+  const MatDesc md = a.mats[mat];
+  const GroupDesc& gd = a.groups[md.group];
+  if (gd.small) return;
+  const int64_t n = md.n, m = md.m;
+  const int64_t col_tiles = (m + kEwCols - 1) / kEwCols;
+  const int64_t local = tile - md.ew_tile_begin;
+  const int64_t row0 = (local / col_tiles) * kEwRows;
+  const int64_t col0 = (local % col_tiles) * kEwCols;
+  const int64_t ldc = gd.ldc;
+  const float* of = reinterpret_cast<const float*>(a.ws + gd.xf_off[a.xf_slot]) +
+                    static_cast<int64_t>(md.index) * gd.r * ldc;
+  const UpdateConsts uc = update_consts_raw(a.lr, a.wd, a.factor[mat], gd.c, kScaleNone);
+
+  if (md.transposed) {
+    // O'(caller i, j) is iterate element (j, i): read iterate rows j, 32
+    // consecutive i per warp access
+    const int w = tid >> 5, lane = tid & 31;
+    const int64_t i = row0 + lane;
+#pragma unroll 4
+    for (int q = 0; q < kEwCols / 8; ++q) {
+      const int cc = w * (kEwCols / 8) + q;
+      const int64_t j = col0 + cc;
+      stage[lane][cc] = (i < n && j < m) ? of[j * ldc + i] : 0.f;
+    }
+    __syncthreads();
+  }
+  // caller element (row, col): thread -> one column, rows (tid / 128) + 2 k
+  constexpr int R = kEwRows / 2;
+  const int cc = tid & (kEwCols - 1);
+  const int64_t col = col0 + cc;
+  float o[R], w[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const int rr = (tid >> 7) + 2 * k;
+    const int64_t row = row0 + rr;
+    const bool in = row < n && col < m;
+    o[k] = !in ? 0.f : (md.transposed ? stage[rr][cc] : of[row * ldc + col]);
+    w[k] = (in && md.W) ? md.W[row * m + col] : 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const int64_t row = row0 + (tid >> 7) + 2 * k;
+    if (row >= n || col >= m) continue;
+    if (md.O) md.O[row * m + col] = o[k];
+    if (md.W) md.W[row * m + col] = fmaf(w[k], uc.keep, -uc.step * o[k]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rms_reduce(const FinishArgs& args, cudaStream_t stream) {
+  if (args.nmats <= 0) return cudaSuccess;
+  rms_reduce_kernel<<<args.nmats, 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finish(const FinishArgs& args, cudaStream_t stream) {
+  if (args.total_tiles <= 0) return cudaSuccess;
+  if (args.total_tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  finish_kernel<<<static_cast<unsigned>(args.total_tiles), 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

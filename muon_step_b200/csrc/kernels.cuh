@@ -21,6 +21,11 @@ cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid,
 // per matrix (bf16 precision).
 cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream);
 
+// Unit-RMS update scale, grouped / fp32 path: per-matrix RMS of O' from the
+// last Apply's sums of squares, then W <- W (1 - lr wd) - lr (gamma / RMS) O'.
+cudaError_t launch_rms_reduce(const FinishArgs& args, cudaStream_t stream);
+cudaError_t launch_finish(const FinishArgs& args, cudaStream_t stream);
+
 // The same stage in fp32 on the CUDA cores (validation precision).
 cudaError_t launch_stage_simt(StageKind kind, const StageArgs& args, int grid,
                               cudaStream_t stream);

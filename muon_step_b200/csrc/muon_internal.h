@@ -103,6 +103,9 @@ struct StageArgs {
   int32_t xsrc;           // which ping-pong buffer holds the current iterate
   float a, b, c;          // this step's coefficients
   float lr, wd, gamma;    // update hyper-parameters (last step)
+  int32_t scale_mode;     // muon_scale_mode_t of the update
+  int32_t sumsq_per_tile; // > 0: also record sums of squares of X' (per tile slots)
+  float* sumsq;           // ... into sumsq[tile * sumsq_per_tile + slot]
   uint64_t wait_limit_ns; // bound on every spin-wait
 };
 
@@ -136,8 +139,26 @@ struct SmallArgs {
   int64_t nsmall;
   int32_t steps;
   float lr, wd, gamma;    // update hyper-parameters
+  int32_t scale_mode;     // muon_scale_mode_t of the update
   uint64_t wait_limit_ns;
   float abc[kMaxSteps * 3];
+};
+
+// Update pass of the unit-RMS scale mode (matrices on the grouped or fp32
+// path): W <- W keep - lr factor[mat] O', O' read from the fp32 iterate.
+struct FinishArgs {
+  const GroupDesc* groups;
+  const MatDesc* mats;
+  const int32_t* tile_mat;  // elementwise tiling of the caller matrices
+  char* ws;
+  const float* sumsq;       // per-tile slots of sum of squares of O'
+  float* factor;            // per matrix gamma / RMS(O') (0 when O' = 0)
+  int64_t total_tiles;      // elementwise tiles
+  int32_t nmats;
+  int32_t xf_slot;          // which fp32 iterate buffer holds O'
+  int32_t sumsq_per_tile;
+  int32_t apply_kind;       // tile table the sums were recorded on
+  float lr, wd, gamma;
 };
 
 // error bits in the device error word

@@ -16,6 +16,7 @@ template <int KIND>
 __global__ void __launch_bounds__(256) stage_simt_kernel(const __grid_constant__ StageArgs a) {
   __shared__ __align__(16) float As[kSBK][kSBM + 4];
   __shared__ __align__(16) float Bs[kSBK][kSBN + 4];
+  __shared__ float red[8];
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;
 
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(256) stage_simt_kernel(const __grid_constant__
     float* xnext = reinterpret_cast<float*>(a.ws + gd.xf_off[a.xsrc ^ 1]) + b * r * ldc;
     float* Aw = reinterpret_cast<float*>(a.ws + gd.a_off) + b * r * ldr;
     float* Bw = reinterpret_cast<float*>(a.ws + gd.b_off) + b * r * ldr;
+    float ssq = 0.f;  // sum of squares of X' over this tile (unit-RMS update scale)
 #pragma unroll
     for (int ii = 0; ii < 4; ++ii) {
       const int64_t row = row0 + ty * 4 + ii;
@@ -105,8 +107,21 @@ __global__ void __launch_bounds__(256) stage_simt_kernel(const __grid_constant__
           const float x = s * fmaf(a.a, xcur[row * ldc + col], v);
           if (a.last) write_update(md, uc, row, col, x);
           else xnext[row * ldc + col] = x;
+          ssq = fmaf(x, x, ssq);
         }
       }
+    }
+    if (KIND == kApply && a.sumsq_per_tile > 0) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+      if ((tid & 31) == 0) red[tid >> 5] = ssq;
+      __syncthreads();
+      if (tid == 0) {
+        float tot = 0.f;
+        for (int w = 0; w < 8; ++w) tot += red[w];
+        a.sumsq[t] = tot;
+      }
+      __syncthreads();
     }
   }
 }

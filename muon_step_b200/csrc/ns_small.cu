@@ -75,6 +75,7 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const fl
 
 __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant__ SmallArgs a) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ float red[4];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Xs = base;
   uint8_t* As = Xs + kTileBytes;
@@ -233,9 +234,26 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
     float* T = reinterpret_cast<float*>(As);
 #pragma unroll
     for (int e = 0; e < kS; ++e) T[tid * kS + (e ^ (tid & 31))] = x[e];
+    if (a.scale_mode == kScaleUnitRms) {
+      // RMS(O') over the matrix (zeros outside it), in a fixed order
+      float ssq = 0.f;
+#pragma unroll
+      for (int e = 0; e < kS; ++e) ssq = fmaf(x[e], x[e], ssq);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+      if ((tid & 31) == 0) red[warp] = ssq;
+    }
     __syncthreads();
     {
-      const UpdateConsts uc = update_consts_raw(a.lr, a.wd, a.gamma, c);
+      // unit-RMS: O = O' gamma / RMS(O'), a plain scale once RMS is known
+      float gam = a.gamma;
+      int mode = a.scale_mode;
+      if (mode == kScaleUnitRms) {
+        const float rms = sqrtf((red[0] + red[1] + red[2] + red[3]) / (static_cast<float>(r) * c));
+        gam = rms > 0.f ? a.gamma / rms : 0.f;
+        mode = kScaleNone;
+      }
+      const UpdateConsts uc = update_consts_raw(a.lr, a.wd, gam, c, mode);
       const int lane = tid & 31;
       const bool tr = md.transposed != 0;
       const int rows = tr ? c : r;  // caller rows

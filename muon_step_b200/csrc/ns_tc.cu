@@ -271,13 +271,20 @@ __device__ __forceinline__ void apply_values(const StageArgs& a, float alpha, co
 }
 
 // Apply: write the new fp32 iterate and its bf16 operand copy.
+// `ssq` accumulates this lane's sum of squares of the new iterate (used by
+// the unit-RMS update scale on the last step).
 __device__ __forceinline__ void epi_apply(const StageArgs& a, const GroupDesc& gd, const TileCoord& tc,
                                           int row0, int col0, uint8_t* slot, const float (&v)[32],
-                                          int lane) {
+                                          int lane, float& ssq) {
   const int mat = gd.first_mat + static_cast<int>(tc.b);
   const float alpha = a.first ? a.scale[mat] : 1.f;
   float x[32];
   apply_values(a, alpha, slot, v, lane, x);
+  if (a.sumsq_per_tile > 0) {
+    // rows and columns past the matrix hold zeros (zero-filled operands)
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ssq = fmaf(x[e], x[e], ssq);
+  }
 #pragma unroll
   for (int q = 0; q < 8; ++q)
     *reinterpret_cast<float4*>(slot + sw128_chunk(lane, q)) =
@@ -581,6 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
       const int bz = static_cast<int>(tc.b);
       const int mat = gd.first_mat + bz;
       const void* in_map = tmap(a, tc.g, C::kApplyLike ? kTmXfE : kTmAE);
+      float ssq = 0.f;  // sum of squares of this warp's share of X' (unit-RMS scale)
       // the last step also brings the weight chunk, in the caller's orientation
       bool w_in = false;
       bool w_tr = false;
@@ -639,7 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
         }
         if (live) {
           if (KIND == kApply) {
-            epi_apply(a, gd, tc, row0, col0, slot, v, lane);
+            epi_apply(a, gd, tc, row0, col0, slot, v, lane, ssq);
           } else if (KIND == kApplyLast) {
             epi_apply_last(a, gd, tc, row0, col0, slot, v, lane);
           } else {
@@ -651,6 +659,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
         // group" always means "the chunk that used the other slot"
         __syncwarp();
         if (lane == 0) ptx::bulk_commit();
+      }
+      if (KIND == kApply && a.sumsq_per_tile > 0) {
+        // one slot per (tile, CTA of the pair, epilogue warp); every slot is written
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+        if (lane == 0) a.sumsq[(t * 2 + rank) * kEpiWarps + ew] = ssq;
       }
       ptx::tc_fence_before();
       __syncwarp();

@@ -41,15 +41,21 @@ struct UpdateConsts {
   float step;  // lr gamma sqrt(max(n, m))
 };
 
-__device__ __forceinline__ UpdateConsts update_consts_raw(float lr, float wd, float gamma, int c) {
+// Scale modes of the update (muon_scale_mode_t).
+enum : int { kScaleShape = 0, kScaleUnitRms = 1, kScaleNone = 2 };
+
+// step = lr gamma sqrt(max(n, m)) (shape), lr gamma (none); the unit-RMS mode
+// passes gamma / RMS(O') as `gamma` with the none rule.
+__device__ __forceinline__ UpdateConsts update_consts_raw(float lr, float wd, float gamma, int c,
+                                                          int scale_mode = kScaleShape) {
   UpdateConsts u;
   u.keep = 1.0f - lr * wd;
-  u.step = lr * gamma * sqrtf(static_cast<float>(c));
+  u.step = (scale_mode == kScaleShape) ? lr * gamma * sqrtf(static_cast<float>(c)) : lr * gamma;
   return u;
 }
 
 __device__ __forceinline__ UpdateConsts update_consts(const StageArgs& a, int c) {
-  return update_consts_raw(a.lr, a.wd, a.gamma, c);
+  return update_consts_raw(a.lr, a.wd, a.gamma, c, a.scale_mode);
 }
 
 __device__ __forceinline__ void write_update(const MatDesc& md, const UpdateConsts& u,

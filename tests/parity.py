@@ -38,7 +38,8 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / nb)
 
 
-def run_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1):
+def run_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1,
+             scale_mode="shape"):
     """Snapshot the sampled inputs, run `steps` Muon steps through the library
     (plan API) capturing O', and return per-sample records."""
     import muon_step_b200 as ms
@@ -49,7 +50,7 @@ def run_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps
                   wl.M[k].double().cpu().numpy()) for k in idx}
     O = {k: torch.empty_like(wl.W[k]) for k in idx}
     params = [(wl.W[k], wl.G[k], wl.M[k], O.get(k)) for k in range(wl.count)]
-    plan = ms.MuonPlan(params, precision=precision, schedule=schedule)
+    plan = ms.MuonPlan(params, precision=precision, schedule=schedule, scale_mode=scale_mode)
     ws = plan.alloc_workspace()
     history = []
     for _ in range(steps):
@@ -62,9 +63,11 @@ def run_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps
     return before, after, history, hyper
 
 
-def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1):
+def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, steps=1,
+               scale_mode="shape"):
     """Compare the library's step(s) with the oracle; return worst errors."""
-    before, after, history, hyper = run_step(wl, precision, hyper, schedule, sample, steps)
+    before, after, history, hyper = run_step(wl, precision, hyper, schedule, sample, steps,
+                                             scale_mode)
     sched = muon_oracle.HYBRID_SCHEDULE if schedule is None else schedule
     worst = {"O": 0.0, "O_over_tol": 0.0, "M": 0.0, "W_given_O": 0.0, "W": 0.0}
     for k, (W, G, M) in before.items():
@@ -72,7 +75,8 @@ def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, ste
         for s in range(steps):
             W, M, O_ref = muon_oracle.muon_step(W, G, M, lr=hyper["lr"], mu=hyper["mu"],
                                                 wd=hyper["wd"], gamma=hyper["gamma"],
-                                                nesterov_on=hyper["nesterov"], schedule=sched)
+                                                nesterov_on=hyper["nesterov"], schedule=sched,
+                                                scale_mode=scale_mode)
             e = rel(history[s][k], O_ref)
             worst["O"] = max(worst["O"], e)
             worst["O_over_tol"] = max(worst["O_over_tol"], e / tol_o(precision, (n, m)))
@@ -82,8 +86,14 @@ def check_step(wl, precision="bf16", hyper=None, schedule=None, sample=None, ste
         if steps == 1:
             # the update arithmetic, given the library's own O'
             W0 = before[k][0]
-            W_from_O = muon_oracle.decay_and_update(
-                W0, muon_oracle.rescale(history[0][k], n, m, hyper["gamma"]), hyper["lr"], hyper["wd"])
+            O_gpu = history[0][k]
+            if scale_mode == "shape":
+                O_sc = muon_oracle.rescale(O_gpu, n, m, hyper["gamma"])
+            elif scale_mode == "unit_rms":
+                O_sc = muon_oracle.rescale_unit_rms(O_gpu, hyper["gamma"])
+            else:
+                O_sc = muon_oracle.rescale_none(O_gpu, hyper["gamma"])
+            W_from_O = muon_oracle.decay_and_update(W0, O_sc, hyper["lr"], hyper["wd"])
             worst["W_given_O"] = max(worst["W_given_O"], rel(W_gpu, W_from_O))
     return worst
 

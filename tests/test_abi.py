@@ -136,6 +136,16 @@ def expected_workspace(shapes, prec):
     off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
+    # unit-RMS scale: sums of squares per Apply tile (8 slots on tensor cores), a factor per matrix
+    if prec == MUON_NS_BF16:
+        apply_tiles = sum(len(mem) * math.ceil(r / 256) * math.ceil(c / 256)
+                          for (r, c), mem in groups.items() if c > 128)
+        slots = 8
+    else:
+        apply_tiles = sum(len(mem) * math.ceil(r / 64) * math.ceil(c / 64) for (r, c), mem in groups.items())
+        slots = 1
+    off = al(off + apply_tiles * slots * 4, 256)
+    off = al(off + nm * 4, 256)
     off = al(off, 1024)
     for (r, c), mem in sorted(groups.items(), key=lambda kv: order.index(kv[0])):
         k = len(mem)
@@ -185,6 +195,37 @@ def test_launch_list(lib):
     assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 5] + grouped
     # the fp32 validation precision has no small-matrix kernel
     assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + grouped
+
+
+def test_scale_modes_change_the_launch_list(lib):
+    st, plan = create(lib, [(64, 64), (300, 400)])
+    cnt = ctypes.c_int()
+    kinds = (ctypes.c_int * 128)()
+
+    def kinds_now():
+        assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 128) == MUON_OK
+        return list(kinds[:cnt.value])
+
+    shape = kinds_now()
+    assert shape[-1] == 4
+    # unit-RMS: the last Apply keeps O', then a per-matrix reduction and an update pass
+    assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
+    assert kinds_now() == shape[:-1] + [3, 6, 7]
+    assert lib.muon_plan_set_scale_mode(plan, 2) == MUON_OK
+    assert kinds_now() == shape
+    assert lib.muon_plan_set_scale_mode(plan, 3) == MUON_ERR_INVALID_ARG
+    lib.muon_plan_destroy(plan)
+    # small matrices only: the small-matrix kernel reduces on chip
+    st, plan = create(lib, [(64, 64)])
+    assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
+    assert kinds_now() == [0, 5]
+    lib.muon_plan_destroy(plan)
+    # orthogonalisation plans have no update to scale
+    ns = ctypes.c_void_p()
+    mats = (MuonNsMatrix * 1)(MuonNsMatrix(FAKE, 2 * FAKE, 5, 9))
+    assert lib.muon_plan_create_ns(mats, 1, MUON_NS_BF16, None, ctypes.byref(ns)) == MUON_OK
+    assert lib.muon_plan_set_scale_mode(ns, 1) == MUON_ERR_INVALID_ARG
+    lib.muon_plan_destroy(ns)
 
 
 def test_flops_count_the_computed_tiles(lib):

@@ -193,3 +193,16 @@ def test_distributed_step_world_one_matches_plan():
             assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k])
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("scale_mode", ["unit_rms", "none"])
+def test_scale_modes(precision, scale_mode):
+    """Unit-RMS and no-rescale updates on small, large, transposed and
+    unaligned matrices (small-matrix kernel, grouped kernels, update pass)."""
+    shapes = [(64, 64), (100, 37), (300, 520), (520, 300), (257, 129), (1, 7)]
+    wl = workloads.make_random(shapes, device="cuda", seed=29)
+    hyper = dict(wl.hyper, gamma=0.2 if scale_mode == "unit_rms" else 1.0)
+    worst = check_step(wl, precision, hyper=hyper, scale_mode=scale_mode)
+    assert worst["O_over_tol"] <= 1.0, worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
