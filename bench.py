@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
+    ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
     return ap.parse_args()
 
 
@@ -66,10 +67,10 @@ def metric_flops(shapes, ns_steps=10):
 
 
 def apply_bytes(shapes):
-    """Algorithmic HBM bytes of one Apply launch: B (bf16 r x r) and X (bf16
-    r x c) operands read once, fp32 iterate read and written, bf16 iterate
-    written: 2 r^2 + 12 r c per matrix."""
-    return sum(2.0 * min(n, m) ** 2 + 12.0 * min(n, m) * max(n, m) for n, m in shapes)
+    """Algorithmic HBM bytes of one Apply launch: B (bf16 r x r) read once, the
+    iterate (bf16 high + low parts, r x c) read once and written once:
+    2 r^2 + 8 r c per matrix."""
+    return sum(2.0 * min(n, m) ** 2 + 8.0 * min(n, m) * max(n, m) for n, m in shapes)
 
 
 def max_over_ranks(x, device, world):
@@ -202,6 +203,50 @@ def traffic_from_profile(config):
     if not m or not h or h.group(1) != kernel_source_hash():
         return None
     return float(m.group(1))
+
+
+ADAMW_VOCAB = 32000
+
+
+def time_adamw_companion(wl, steps, dev, stream, peaks, world):
+    """The AdamW group a model with these matrices would carry: an embedding
+    and a prediction head of ADAMW_VOCAB rows by the model width (the most
+    common matrix dimension), plus two norm vectors per matrix. One launch per
+    step, timed with CUDA events over `steps` steps; HBM-bound, 28 B/element."""
+    import muon_step_b200 as ms
+
+    dims = {}
+    for n, m in wl.shapes:
+        for d in (n, m):
+            dims[d] = dims.get(d, 0) + 1
+    width = max(dims, key=lambda d: (dims[d], -d))
+    sizes = [ADAMW_VOCAB * width, ADAMW_VOCAB * width] + [width] * (2 * wl.count)
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    tensors = []
+    for n in sizes:
+        p = torch.randn(n, generator=gen, device=dev) * 0.02
+        g = torch.randn(n, generator=gen, device=dev) * 1e-3
+        tensors.append((p, g, torch.zeros_like(p), torch.zeros_like(p)))
+    plan = ms.AdamWPlan(tensors)
+    ws = plan.alloc_workspace()
+    for t in range(1, 4):
+        plan.execute(ws, step=t, stream=stream)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(4, 4 + steps):
+        plan.execute(ws, step=t, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    t_ms = max_over_ranks(e0.elapsed_time(e1), dev, world) / steps
+    elems = plan.numel
+    gbs = 28.0 * elems / (t_ms / 1e3) / 1e9
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"elements": elems, "tensors": len(sizes), "width": width, "vocab": ADAMW_VOCAB,
+            "ms_per_step": t_ms, "achieved_gbs": gbs, "frac_hbm": gbs / hbm,
+            "bytes_per_element": 28, "gpu_launches_per_step": 1}
 
 
 def run_reference(args, rank, world):
@@ -426,6 +471,11 @@ def main():
                "ms_per_step": te / args.steps}
         assert ms.sync_status() == 0
 
+    # ---- AdamW companion group (separate timed region; not part of `value`)
+    adamw = None
+    if not args.no_adamw:
+        adamw = time_adamw_companion(wl, args.steps, dev, stream, peaks, world)
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -460,6 +510,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "companion_adamw": adamw,
         }
         print(json.dumps(line), flush=True)
     del graph

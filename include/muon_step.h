@@ -64,7 +64,8 @@ typedef enum {
 } muon_status_t;
 
 /* Newton-Schulz operand precision. BF16: bf16 tensor-core operands with fp32
- * accumulation and an fp32 master copy of the iterate. FP32: fp32 operands on
+ * accumulation; the iterate is kept as bf16 high + low parts (16 significant
+ * bits) so that the a X term does not lose the operand's rounding. FP32: fp32 operands on
  * the CUDA cores (validation; slow). Momentum and update are fp32 in both. */
 typedef enum { MUON_NS_BF16 = 0, MUON_NS_FP32 = 1 } muon_precision_t;
 
@@ -136,6 +137,18 @@ MUON_API muon_status_t muon_plan_create_ns(const muon_ns_matrix_t* mats, int cou
  * UNIT_RMS mode the last step adds a per-matrix reduction and an elementwise
  * update pass for matrices larger than 128 x 128. */
 MUON_API muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode);
+
+/* Per-matrix diagnostics of later executes ([V4-breakdown] section
+ * "更新尺度：让 Muon 借用 AdamW 的超参": the update-RMS lemma says RMS(O') is
+ * about sqrt(1 / max(n, m)), so the shape rule's update has RMS about gamma).
+ * `out` is a caller-owned DEVICE array of 2 * count floats, in the order of
+ * the plan's params; each execute writes
+ *   out[2 i]     = ||N_i||_F   the Frobenius norm of the orthogonaliser's input
+ *   out[2 i + 1] = RMS(O_i)    the RMS of the scaled update that lr multiplies
+ * (0 for a zero gradient). NULL turns them off (the default). With the SHAPE
+ * or NONE scale the last step then adds one per-matrix reduction launch for
+ * matrices larger than 128 x 128. Muon-step plans only. */
+MUON_API muon_status_t muon_plan_set_diagnostics(muon_plan_t plan, float* out);
 
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */
 MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes);

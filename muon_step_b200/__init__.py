@@ -21,11 +21,12 @@ from typing import Iterable, Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import (MUON_ERR_TIMEOUT, MUON_NS_BF16, MUON_NS_FP32, MUON_OK, MuonHyper, MuonNsMatrix,
-                   MuonNsSchedule, MuonParam)
+from ._lib import (MUON_ERR_TIMEOUT, MUON_NS_BF16, MUON_NS_FP32, MUON_OK, AdamwHyper, AdamwParam,
+                   MuonHyper, MuonNsMatrix, MuonNsSchedule, MuonParam)
 
-__all__ = ["MuonError", "MuonPlan", "NsPlan", "muon_step", "ns_orthogonalize", "sync_status",
-           "library", "HYBRID_SCHEDULE", "wait_probe", "set_wait_limit_ns"]
+__all__ = ["MuonError", "MuonPlan", "NsPlan", "AdamWPlan", "muon_step", "ns_orthogonalize",
+           "adamw_step", "sync_status", "library", "HYBRID_SCHEDULE", "wait_probe",
+           "set_wait_limit_ns"]
 
 # the pages' hybrid schedule: 8 aggressive steps, then 2 standard ones
 HYBRID_SCHEDULE = ((3.4445, -4.7750, 2.0315),) * 8 + ((2.0, -1.5, 0.5),) * 2
@@ -84,10 +85,12 @@ def _stream_ptr(stream) -> Optional[int]:
 
 class _PlanBase:
     _plan = None
+    _destroy = None
 
     def __del__(self):
-        if self._plan:
-            _lib.load().muon_plan_destroy(self._plan)
+        # the destroy function is bound at creation: module globals may be gone at exit
+        if self._plan and self._destroy is not None:
+            self._destroy(self._plan)
             self._plan = None
 
     @property
@@ -173,6 +176,7 @@ class MuonPlan(_PlanBase):
                                             ctypes.byref(sched) if sched else None,
                                             ctypes.byref(plan)), "muon_plan_create")
         self._plan = plan
+        self._destroy = _lib.load().muon_plan_destroy
         if scale_mode != "shape":
             self.set_scale_mode(scale_mode)
 
@@ -184,6 +188,23 @@ class MuonPlan(_PlanBase):
         again afterwards (the launch list may change)."""
         _check(_lib.load().muon_plan_set_scale_mode(self._plan, self.SCALE_MODES[mode]),
                "muon_plan_set_scale_mode")
+
+    def set_diagnostics(self, out: Optional[torch.Tensor]):
+        """Write per-matrix diagnostics on every later execute into `out`, a
+        float32 CUDA tensor of shape (count, 2): column 0 = ||N||_F (the
+        orthogonaliser's input), column 1 = RMS of the scaled update O. None
+        turns them off. Timing events must be set again afterwards."""
+        if out is None:
+            ptr = None
+        else:
+            count = len(self._tensors)
+            if (out.dtype != torch.float32 or not out.is_cuda or not out.is_contiguous()
+                    or out.numel() != 2 * count or out.device != self.device):
+                raise ValueError(f"diagnostics need a contiguous float32 tensor of {2 * count} "
+                                 f"elements on {self.device}")
+            ptr = out.data_ptr()
+        _check(_lib.load().muon_plan_set_diagnostics(self._plan, ptr), "muon_plan_set_diagnostics")
+        self._diag = out
 
     def execute(self, workspace=None, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2,
                 nesterov=True, stream=None):
@@ -217,6 +238,7 @@ class NsPlan(_PlanBase):
                                                ctypes.byref(sched) if sched else None,
                                                ctypes.byref(plan)), "muon_plan_create_ns")
         self._plan = plan
+        self._destroy = _lib.load().muon_plan_destroy
 
     def execute(self, workspace=None, stream=None):
         workspace = self._ws(workspace)
@@ -270,6 +292,108 @@ def ns_orthogonalize(xs, out=None, precision="bf16", schedule=None, eps=None, wo
                                 workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
            "ns_orthogonalize")
     return out
+
+
+def _flat(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous float32 tensor")
+    return t
+
+
+def _adamw_items(params):
+    items, keep = [], []
+    for k, q in enumerate(params):
+        p, g, m, v = (_flat(t, f"params[{k}].{nm}") for t, nm in zip(q, "pgmv"))
+        if not (p.numel() == g.numel() == m.numel() == v.numel()):
+            raise ValueError(f"params[{k}]: p, g, m, v must have one size")
+        items.append(AdamwParam(p.data_ptr(), g.data_ptr(), m.data_ptr(), v.data_ptr(), p.numel()))
+        keep.append((p, g, m, v))
+    if not items:
+        raise ValueError("no tensors")
+    return (AdamwParam * len(items))(*items), keep
+
+
+def _adamw_hyper(lr, betas, eps, weight_decay, step, step_tensor):
+    if step_tensor is not None:
+        if (step_tensor.dtype != torch.int32 or not step_tensor.is_cuda
+                or step_tensor.numel() != 1):
+            raise TypeError("step_tensor must be a one-element int32 CUDA tensor")
+        return AdamwHyper(lr=lr, eps=eps, weight_decay=weight_decay, step=0, beta1=betas[0],
+                          beta2=betas[1], step_dev=step_tensor.data_ptr())
+    return AdamwHyper(lr=lr, eps=eps, weight_decay=weight_decay, step=int(step), beta1=betas[0],
+                      beta2=betas[1], step_dev=None)
+
+
+class AdamWPlan:
+    """A planned AdamW step over a fixed list of (p, g, m, v) float32 CUDA
+    tensors (any shape, contiguous; m and v are the moment buffers, zero at
+    the start). One kernel launch per execute (C ABI muon_adamw_plan_*)."""
+
+    _plan = None
+    _destroy = None
+
+    def __init__(self, params: Iterable):
+        arr, self._tensors = _adamw_items(params)
+        self.device = self._tensors[0][0].device
+        lib = _lib.load()
+        plan = ctypes.c_void_p()
+        _check(lib.muon_adamw_plan_create(arr, len(arr), ctypes.byref(plan)), "muon_adamw_plan_create")
+        self._plan = plan
+        self._destroy = lib.muon_adamw_plan_destroy
+        self._ws_cache = None
+
+    def __del__(self):
+        if self._plan and self._destroy is not None:
+            self._destroy(self._plan)
+            self._plan = None
+
+    @property
+    def workspace_bytes(self) -> int:
+        n = ctypes.c_size_t()
+        _check(_lib.load().muon_adamw_plan_workspace_size(self._plan, ctypes.byref(n)),
+               "muon_adamw_plan_workspace_size")
+        return n.value
+
+    @property
+    def numel(self) -> int:
+        n = ctypes.c_int64()
+        _check(_lib.load().muon_adamw_plan_numel(self._plan, ctypes.byref(n)), "muon_adamw_plan_numel")
+        return n.value
+
+    def alloc_workspace(self, device=None) -> torch.Tensor:
+        device = self.device if device is None else device
+        return torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8, device=device)
+
+    def execute(self, workspace=None, lr=0.02, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
+                step=1, step_tensor=None, stream=None):
+        """One AdamW step at step number `step` (from 1), or at the number held
+        on the device in `step_tensor` (int32, read by the kernel)."""
+        if workspace is None:
+            if self._ws_cache is None:
+                self._ws_cache = self.alloc_workspace()
+            workspace = self._ws_cache
+        h = _adamw_hyper(lr, betas, eps, weight_decay, step, step_tensor)
+        _check(_lib.load().muon_adamw_plan_execute(self._plan, ctypes.byref(h), workspace.data_ptr(),
+                                                   workspace.numel(), _stream_ptr(stream)),
+               "muon_adamw_plan_execute")
+
+
+def adamw_step(params, step, lr=0.02, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.1,
+               workspace=None, stream=None):
+    """One-shot AdamW step (C ABI muon_adamw_step) over a list of (p, g, m, v)."""
+    arr, keep = _adamw_items(params)
+    lib = _lib.load()
+    if workspace is None:
+        n = ctypes.c_size_t()
+        _check(lib.muon_adamw_workspace_size(arr, len(arr), ctypes.byref(n)),
+               "muon_adamw_workspace_size")
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=keep[0][0].device)
+    h = _adamw_hyper(lr, betas, eps, weight_decay, step, None)
+    _check(lib.muon_adamw_step(arr, len(arr), ctypes.byref(h), workspace.data_ptr(),
+                               workspace.numel(), _stream_ptr(stream)), "muon_adamw_step")
+    return workspace
 
 
 def sync_status(stream=None) -> int:

@@ -31,6 +31,10 @@ EXPORTS = (
     "muon_workspace_size", "muon_step", "ns_workspace_size", "ns_orthogonalize",
     "muon_sync_status", "muon_status_string", "muon_abi_version", "muon_set_wait_limit_ns",
     "muon_wait_probe", "muon_step_static_scratch", "muon_plan_set_scale_mode",
+    "muon_plan_set_diagnostics",
+    "muon_adamw_plan_create", "muon_adamw_plan_workspace_size", "muon_adamw_plan_execute",
+    "muon_adamw_plan_numel", "muon_adamw_plan_destroy", "muon_adamw_workspace_size",
+    "muon_adamw_step",
 )
 
 
@@ -47,6 +51,17 @@ class MuonNsSchedule(ctypes.Structure):
 class MuonNsMatrix(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("O", ctypes.c_void_p), ("n", ctypes.c_int64),
                 ("m", ctypes.c_int64)]
+
+
+class AdamwParam(ctypes.Structure):
+    _fields_ = [("p", ctypes.c_void_p), ("g", ctypes.c_void_p), ("m", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("numel", ctypes.c_int64)]
+
+
+class AdamwHyper(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("step", ctypes.c_int32), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("step_dev", ctypes.c_void_p)]
 
 
 class MuonHyper(ctypes.Structure):
@@ -80,6 +95,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_plan_flops": (st, [vp, P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_double)]),
         "muon_plan_destroy": (None, [vp]),
         "muon_plan_set_scale_mode": (st, [vp, ctypes.c_int]),
+        "muon_plan_set_diagnostics": (st, [vp, vp]),
+        "muon_adamw_plan_create": (st, [P(AdamwParam), ctypes.c_int, P(vp)]),
+        "muon_adamw_plan_workspace_size": (st, [vp, P(ctypes.c_size_t)]),
+        "muon_adamw_plan_execute": (st, [vp, P(AdamwHyper), vp, ctypes.c_size_t, vp]),
+        "muon_adamw_plan_numel": (st, [vp, P(ctypes.c_int64)]),
+        "muon_adamw_plan_destroy": (None, [vp]),
+        "muon_adamw_workspace_size": (st, [P(AdamwParam), ctypes.c_int, P(ctypes.c_size_t)]),
+        "muon_adamw_step": (st, [P(AdamwParam), ctypes.c_int, P(AdamwHyper), vp, ctypes.c_size_t,
+                                 vp]),
         "muon_workspace_size": (st, [P(MuonParam), ctypes.c_int, ctypes.c_int, P(ctypes.c_size_t)]),
         "muon_step": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                            ctypes.c_float, ctypes.c_int, P(MuonNsSchedule), ctypes.c_int, vp,

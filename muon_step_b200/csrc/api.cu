@@ -124,6 +124,7 @@ struct muon_plan_s {
   int scale_mode = MUON_SCALE_SHAPE;
   int sumsq_per_tile = 1;           // sum-of-squares slots per Apply tile (unit-RMS scale)
   size_t off_sumsq = 0, off_factor = 0;
+  float* diag = nullptr;            // caller's diagnostics output (2 floats per matrix) or NULL
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -164,6 +165,8 @@ void make_launch_list(muon_plan_s* p) {
     if (unit) {
       p->launch_kinds.push_back(6);
       p->launch_kinds.push_back(7);
+    } else if (p->diag) {
+      p->launch_kinds.push_back(6);  // update-RMS diagnostics of the fused last step
     }
   }
 }
@@ -242,6 +245,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
       md.transposed = md.n > md.m ? 1 : 0;
       md.group = static_cast<int32_t>(g);
       md.index = static_cast<int32_t>(idx);
+      md.caller = static_cast<int32_t>(members[g][idx]);
       // the last step moves W and O by TMA when their rows are 16-byte aligned
       const bool rows16 = (md.m % 4) == 0;
       md.flags = 0;
@@ -290,18 +294,23 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     const size_t x_elems = cnt * static_cast<size_t>(gd.r) * gd.ldc;
     const size_t a_elems = cnt * static_cast<size_t>(gd.r) * gd.ldr;
     const size_t ab_bytes = tc ? 2 : 4;
-    gd.xf_off[0] = static_cast<int64_t>(off);
-    off = align_up(off + x_elems * 4, 1024);
     if (tc) {
-      gd.xf_off[1] = gd.xf_off[0];
+      // bf16 mode: the iterate as high part (ping-pong: the Apply product reads
+      // the current one whole) and low part (updated in place by its owner tile)
+      gd.xf_off[0] = gd.xf_off[1] = 0;
       gd.xb_off[0] = static_cast<int64_t>(off);
       off = align_up(off + x_elems * 2, 1024);
       gd.xb_off[1] = static_cast<int64_t>(off);
       off = align_up(off + x_elems * 2, 1024);
+      gd.xlo_off = static_cast<int64_t>(off);
+      off = align_up(off + x_elems * 2, 1024);
     } else {
+      gd.xf_off[0] = static_cast<int64_t>(off);
+      off = align_up(off + x_elems * 4, 1024);
       gd.xf_off[1] = static_cast<int64_t>(off);
       off = align_up(off + x_elems * 4, 1024);
       gd.xb_off[0] = gd.xb_off[1] = 0;
+      gd.xlo_off = 0;
     }
     gd.a_off = static_cast<int64_t>(off);
     off = align_up(off + a_elems * ab_bytes, 1024);
@@ -345,8 +354,7 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
           encode_bf16_3d(&m[kTmA], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 64, 128, SW128) &&
           encode_bf16_3d(&m[kTmB], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 64, 128, SW128) &&
           // epilogue maps (32 x 32 chunks)
-          encode_3d(&m[kTmXfE], base + gd.xf_off[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.c, gd.r,
-                    gd.ldc, gd.count, 32, 32, SW128) &&
+          encode_bf16_3d(&m[kTmXloE], base + gd.xlo_off, gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
           encode_bf16_3d(&m[kTmXb0E], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
           encode_bf16_3d(&m[kTmXb1E], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
           encode_bf16_3d(&m[kTmAE], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64) &&
@@ -536,9 +544,10 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   ew.nmats = static_cast<int32_t>(plan->mats.size());
   ew.mode = plan->mode;
   ew.nesterov = (plan->mode == 0 && hyper->nesterov) ? 1 : 0;
-  ew.write_bf16 = plan->prec == MUON_NS_BF16 ? 1 : 0;
+  ew.split = plan->prec == MUON_NS_BF16 ? 1 : 0;
   ew.mu = plan->mode == 0 ? hyper->momentum : 0.f;
   ew.eps = plan->eps;
+  ew.diag = plan->mode == 0 ? plan->diag : nullptr;
   if ((st = record(plan, 0, stream)) != MUON_OK) return st;
   if (launch_elementwise(ew, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if ((st = record(plan, 1, stream)) != MUON_OK) return st;
@@ -563,6 +572,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       sm.gamma = hyper->gamma;
     }
     sm.scale_mode = plan->scale_mode;
+    sm.diag = plan->mode == 0 ? plan->diag : nullptr;
     sm.wait_limit_ns = limit;
     for (int k = 0; k < 3 * plan->steps; ++k) sm.abc[k] = plan->abc[k];
     const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
@@ -572,6 +582,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   }
   if (plan->stage_tiles[kApply] == 0) return MUON_OK;
   const bool unit = plan->scale_mode == MUON_SCALE_UNIT_RMS;
+  const bool diag = plan->mode == 0 && plan->diag != nullptr;
   for (int k = 0; k < plan->steps; ++k) {
     for (int kind = 0; kind < kNumKinds; ++kind) {
       StageArgs sa{};
@@ -587,10 +598,11 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       const bool last = k == plan->steps - 1;
       sa.first = k == 0;
       // unit-RMS scale: the last Apply keeps O' and its sums of squares; the
-      // update comes after the per-matrix reduction
+      // update comes after the per-matrix reduction. Diagnostics: the fused
+      // last step records the sums too.
       sa.last = last && !unit;
       sa.scale_mode = plan->scale_mode;
-      if (unit && last && kind == kApply) {
+      if ((unit || diag) && last && kind == kApply) {
         sa.sumsq_per_tile = plan->sumsq_per_tile;
         sa.sumsq = reinterpret_cast<float*>(ws + plan->off_sumsq);
       }
@@ -618,7 +630,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
     }
   }
-  if (unit) {
+  if (unit || diag) {
     FinishArgs fa{};
     fa.groups = groups;
     fa.mats = mats;
@@ -628,19 +640,25 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
     fa.factor = reinterpret_cast<float*>(ws + plan->off_factor);
     fa.total_tiles = plan->ew_tiles;
     fa.nmats = static_cast<int32_t>(plan->mats.size());
-    // fp32 path: the last step wrote buffer (steps & 1); tensor cores update in place
-    fa.xf_slot = tc ? 0 : (plan->steps & 1);
+    // the last step (index steps - 1) wrote iterate buffer (steps & 1): the
+    // fp32 iterate, or the high part of the split bf16 iterate
+    fa.xf_slot = plan->steps & 1;
+    fa.split = tc ? 1 : 0;
     fa.sumsq_per_tile = plan->sumsq_per_tile;
     fa.apply_kind = kApply;
     fa.lr = hyper->lr;
     fa.wd = hyper->weight_decay;
     fa.gamma = hyper->gamma;
+    fa.scale_mode = plan->scale_mode;
+    fa.diag = plan->diag;
     if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
     if (launch_rms_reduce(fa, stream) != cudaSuccess) return MUON_ERR_CUDA;
     if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
-    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
-    if (launch_finish(fa, stream) != cudaSuccess) return MUON_ERR_CUDA;
-    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (unit) {
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      if (launch_finish(fa, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
   }
   return MUON_OK;
 }
@@ -650,6 +668,15 @@ muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode)
   if (mode != MUON_SCALE_SHAPE && mode != MUON_SCALE_UNIT_RMS && mode != MUON_SCALE_NONE)
     return MUON_ERR_INVALID_ARG;
   plan->scale_mode = mode;
+  make_launch_list(plan);
+  plan->events.clear();  // the launch list may have changed: timing must be set again
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_diagnostics(muon_plan_t plan, float* out) {
+  if (!plan || plan->mode != 0) return MUON_ERR_INVALID_ARG;
+  if (out && (reinterpret_cast<uintptr_t>(out) & 3) != 0) return MUON_ERR_INVALID_ARG;
+  plan->diag = out;
   make_launch_list(plan);
   plan->events.clear();  // the launch list may have changed: timing must be set again
   return MUON_OK;
@@ -767,5 +794,8 @@ cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limi
   wait_probe_kernel<<<1, 1, 0, stream>>>(flag, err, limit_ns);
   return cudaGetLastError();
 }
+
+// Current device, checked to be an sm_100 part; sets up the per-device state.
+muon_status_t current_device_checked(int* dev) { return device_setup(dev); }
 
 }  // namespace muon

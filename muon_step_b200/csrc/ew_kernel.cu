@@ -9,10 +9,12 @@
 // Algorithm 1 steps one and two; "Ch 06 · Muon" §5 Algorithm 1 (momentum,
 // Nesterov and the division by ||N_t||_F). The scale s is not applied here:
 // the first Newton-Schulz step folds s^2 into the Gram matrix and s into the
-// iterate, so the unscaled N is written once, in fp32 and as the bf16 operand.
+// iterate, so the unscaled N is written once: in bf16 mode as a bf16 high part
+// (the tensor-core operand) plus a bf16 low part, N = high + low to 16
+// significant bits; in fp32 mode as fp32.
 //
-// HBM-bound: each element reads G and M (8 B) and writes M, the fp32 iterate
-// and the bf16 operand (10 B). Tiles are 32 x 128 elements; a tile's threads
+// HBM-bound: each element reads G and M (8 B) and writes M and the two bf16
+// parts (8 B; fp32 mode: M and the fp32 iterate). Tiles are 32 x 128 elements; a tile's threads
 // read and write whole 128-byte lines. When the iterate is the transpose, the
 // tile is staged in shared memory so that the transposed writes stay
 // coalesced. Per-tile partial sums of squares go to a buffer; the last tile of
@@ -63,8 +65,20 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
 
   const int64_t ldc = gd.ldc;
   const int64_t mat_elems = static_cast<int64_t>(gd.r) * ldc;
+  // fp32 mode: the fp32 iterate; bf16 mode: its bf16 high part (the MMA
+  // operand) and low part, N = high + low to 16 significant bits
   float* xf = reinterpret_cast<float*>(a.ws + gd.xf_off[0]) + md.index * mat_elems;
   __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xb_off[0]) + md.index * mat_elems;
+  __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xlo_off) + md.index * mat_elems;
+  auto put = [&](int64_t xo, float v) {
+    if (a.split) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      xb[xo] = h;
+      xl[xo] = __float2bfloat16_rn(v - __bfloat162float(h));
+    } else {
+      xf[xo] = v;
+    }
+  };
   const bool transposed = md.transposed != 0;
   const float mu = a.mu;
   float sumsq = 0.f;
@@ -113,12 +127,17 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
         sumsq += nv[0] * nv[0] + nv[1] * nv[1] + nv[2] * nv[2] + nv[3] * nv[3];
         if (!transposed) {
           const int64_t xo = row * ldc + col;
-          *reinterpret_cast<float4*>(xf + xo) = make_float4(nv[0], nv[1], nv[2], nv[3]);
-          if (a.write_bf16) {
-            Bf16x4 p;
-            p.lo = __floats2bfloat162_rn(nv[0], nv[1]);
-            p.hi = __floats2bfloat162_rn(nv[2], nv[3]);
-            *reinterpret_cast<Bf16x4*>(xb + xo) = p;
+          if (a.split) {
+            Bf16x4 h, l;
+            h.lo = __floats2bfloat162_rn(nv[0], nv[1]);
+            h.hi = __floats2bfloat162_rn(nv[2], nv[3]);
+            const float2 h01 = __bfloat1622float2(h.lo), h23 = __bfloat1622float2(h.hi);
+            l.lo = __floats2bfloat162_rn(nv[0] - h01.x, nv[1] - h01.y);
+            l.hi = __floats2bfloat162_rn(nv[2] - h23.x, nv[3] - h23.y);
+            *reinterpret_cast<Bf16x4*>(xb + xo) = h;
+            *reinterpret_cast<Bf16x4*>(xl + xo) = l;
+          } else {
+            *reinterpret_cast<float4*>(xf + xo) = make_float4(nv[0], nv[1], nv[2], nv[3]);
           }
         }
       }
@@ -156,9 +175,7 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
         if (a.mode == 0) __stcs(md.M + off, mo);
         sumsq += nv * nv;
         if (!transposed) {
-          const int64_t xo = row * ldc + col;
-          xf[xo] = nv;
-          if (a.write_bf16) xb[xo] = __float2bfloat16_rn(nv);
+          put(row * ldc + col, nv);
         }
       }
       if (transposed) stage[rr][cc] = nv;
@@ -175,10 +192,7 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
       const int cc = w * (kEwCols / 8) + q;
       const int64_t j = col0 + cc;
       if (j < m && i < n) {
-        const float v = stage[lane][cc];
-        const int64_t xo = j * ldc + i;
-        xf[xo] = v;
-        if (a.write_bf16) xb[xo] = __float2bfloat16_rn(v);
+        put(j * ldc + i, stage[lane][cc]);
       }
     }
   }
@@ -211,6 +225,7 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
     double s = 0.0;
     for (int w = 0; w < 8; ++w) s += warp_part_d[w];
     a.scale[mi] = static_cast<float>(1.0 / (sqrt(s) + static_cast<double>(a.eps)));
+    if (a.diag) a.diag[2 * md.caller] = static_cast<float>(sqrt(s));
     a.counter[mi] = 0u;
   }
 }

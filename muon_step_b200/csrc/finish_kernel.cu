@@ -4,7 +4,7 @@
 // "Muon 优化器完全拆解…", section "分布式工程": the Megatron-Bridge recipe scales
 // the update to unit RMS and then by an extra factor, O = gamma O' / RMS(O').
 // RMS(O') needs all of O' before any element of W can move, so here the last
-// Apply stage keeps O' in the fp32 iterate and records sums of squares per
+// Apply stage keeps O' in the iterate buffers and records sums of squares per
 // tile; then
 //
 //   rms_reduce_kernel   one CTA per matrix adds its tiles' sums in a fixed
@@ -15,7 +15,13 @@
 //                       iterate is the transpose, the tile is read through
 //                       shared memory so every global access stays coalesced.
 //
-// HBM-bound: 4 B of O' read, 8 B of W read and written per element.
+// HBM-bound: 4 B of O' read (fp32, or bf16 high + low parts), 8 B of W read
+// and written per element.
+//
+// With diagnostics on, rms_reduce_kernel also runs after a fused last step (any
+// scale mode) and writes the RMS of the applied update per matrix.
+#include <cuda_bf16.h>
+
 #include "kernels.cuh"
 #include "stage_common.cuh"
 
@@ -43,6 +49,14 @@ __global__ void __launch_bounds__(256) rms_reduce_kernel(const __grid_constant__
     for (int w = 0; w < 8; ++w) tot += part[w];
     const double rms = sqrt(tot / (static_cast<double>(md.n) * static_cast<double>(md.m)));
     a.factor[mat] = rms > 0.0 ? static_cast<float>(static_cast<double>(a.gamma) / rms) : 0.f;
+    if (a.diag) {
+      // RMS of the applied update O: gamma sqrt(max(n, m)) RMS(O') (shape), gamma
+      // (unit RMS; 0 when O' = 0) or gamma RMS(O') (none)
+      double o_rms = static_cast<double>(a.gamma) * rms;
+      if (a.scale_mode == kScaleShape) o_rms *= sqrt(static_cast<double>(gd.c));
+      if (a.scale_mode == kScaleUnitRms) o_rms = rms > 0.0 ? static_cast<double>(a.gamma) : 0.0;
+      a.diag[2 * md.caller + 1] = static_cast<float>(o_rms);
+    }
   }
 }
 
@@ -60,8 +74,14 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
   const int64_t row0 = (local / col_tiles) * kEwRows;
   const int64_t col0 = (local % col_tiles) * kEwCols;
   const int64_t ldc = gd.ldc;
-  const float* of = reinterpret_cast<const float*>(a.ws + gd.xf_off[a.xf_slot]) +
-                    static_cast<int64_t>(md.index) * gd.r * ldc;
+  const int64_t mo = static_cast<int64_t>(md.index) * gd.r * ldc;
+  const float* of = reinterpret_cast<const float*>(a.ws + gd.xf_off[a.xf_slot]) + mo;
+  const __nv_bfloat16* oh = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xb_off[a.xf_slot]) + mo;
+  const __nv_bfloat16* ol = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xlo_off) + mo;
+  // O' element at iterate offset k: fp32, or high + low parts
+  auto o_at = [&](int64_t k) -> float {
+    return a.split ? __bfloat162float(oh[k]) + __bfloat162float(ol[k]) : of[k];
+  };
   const UpdateConsts uc = update_consts_raw(a.lr, a.wd, a.factor[mat], gd.c, kScaleNone);
 
   if (md.transposed) {
@@ -73,7 +93,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
     for (int q = 0; q < kEwCols / 8; ++q) {
       const int cc = w * (kEwCols / 8) + q;
       const int64_t j = col0 + cc;
-      stage[lane][cc] = (i < n && j < m) ? of[j * ldc + i] : 0.f;
+      stage[lane][cc] = (i < n && j < m) ? o_at(j * ldc + i) : 0.f;
     }
     __syncthreads();
   }
@@ -87,7 +107,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
     const int rr = (tid >> 7) + 2 * k;
     const int64_t row = row0 + rr;
     const bool in = row < n && col < m;
-    o[k] = !in ? 0.f : (md.transposed ? stage[rr][cc] : of[row * ldc + col]);
+    o[k] = !in ? 0.f : (md.transposed ? stage[rr][cc] : o_at(row * ldc + col));
     w[k] = (in && md.W) ? md.W[row * m + col] : 0.f;
   }
 #pragma unroll

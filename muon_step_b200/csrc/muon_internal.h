@@ -50,7 +50,7 @@ enum TmapSlot : int {
   kTmA = 4,      // Gram matrix A, box {64, 128}
   kTmB = 5,      // polynomial B = bA + cA^2, box {64, 128}
   // epilogue maps, box {32, 32}: loads and stores of one warp's 32 x 32 chunk
-  kTmXfE = 6,    // fp32 iterate, 128-byte swizzle
+  kTmXloE = 6,   // bf16 low part of the iterate, 64-byte swizzle
   kTmXb0E = 7,   // bf16 iterate buffer 0, 64-byte swizzle
   kTmXb1E = 8,   // bf16 iterate buffer 1, 64-byte swizzle
   kTmAE = 9,     // A, 64-byte swizzle
@@ -65,8 +65,9 @@ struct GroupDesc {
   int32_t first_mat;     // internal index of the group's first matrix
   int32_t small;         // 1: runs in the small-matrix kernel, no stage tiles
   int32_t pad0;
-  int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate (fp32 mode ping-pongs)
-  int64_t xb_off[2];     // bf16 iterate, ping-pong
+  int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate, ping-pong (fp32 mode)
+  int64_t xb_off[2];     // bf16 iterate (bf16 mode: its high part, the MMA operand), ping-pong
+  int64_t xlo_off;       // bf16 mode: low part, iterate = high + low (updated in place)
   int64_t a_off, b_off;  // A = X X^T and B = bA + cA^2 (bf16, or fp32 in fp32 mode)
   int64_t tiles_per_mat[kNumKinds];
   int64_t tile_base[kNumKinds];
@@ -83,6 +84,8 @@ struct MatDesc {
   int32_t group;         // shape group
   int32_t index;         // index within the group
   int32_t flags;         // kMatWTma / kMatOTma: W / O reachable by TMA (16-byte rows)
+  int32_t caller;        // position in the caller's list (diagnostics output)
+  int32_t pad1;
   int64_t ew_tile_begin; // first elementwise tile of this matrix
   int64_t ew_tiles;      // number of elementwise tiles
 };
@@ -104,7 +107,7 @@ struct StageArgs {
   float a, b, c;          // this step's coefficients
   float lr, wd, gamma;    // update hyper-parameters (last step)
   int32_t scale_mode;     // muon_scale_mode_t of the update
-  int32_t sumsq_per_tile; // > 0: also record sums of squares of X' (per tile slots)
+  int32_t sumsq_per_tile; // > 0: the last step records sums of squares of X' (per tile slots)
   float* sumsq;           // ... into sumsq[tile * sumsq_per_tile + slot]
   uint64_t wait_limit_ns; // bound on every spin-wait
 };
@@ -123,8 +126,9 @@ struct EwArgs {
   int32_t nmats;
   int32_t mode;           // 0: Muon (momentum + Nesterov), 1: plain normalisation of G
   int32_t nesterov;
-  int32_t write_bf16;     // bf16 mode writes the bf16 operand copy too
+  int32_t split;          // bf16 mode: the iterate as bf16 high + low parts (else fp32)
   float mu, eps;
+  float* diag;            // optional: diag[2 caller] = ||N||_F
 };
 
 // Small-matrix kernel arguments (one CTA per matrix, every step on chip).
@@ -141,11 +145,12 @@ struct SmallArgs {
   float lr, wd, gamma;    // update hyper-parameters
   int32_t scale_mode;     // muon_scale_mode_t of the update
   uint64_t wait_limit_ns;
+  float* diag;            // optional: diag[2 caller + 1] = RMS of the applied update O
   float abc[kMaxSteps * 3];
 };
 
 // Update pass of the unit-RMS scale mode (matrices on the grouped or fp32
-// path): W <- W keep - lr factor[mat] O', O' read from the fp32 iterate.
+// path): W <- W keep - lr factor[mat] O', O' read from the iterate buffers.
 struct FinishArgs {
   const GroupDesc* groups;
   const MatDesc* mats;
@@ -155,10 +160,13 @@ struct FinishArgs {
   float* factor;            // per matrix gamma / RMS(O') (0 when O' = 0)
   int64_t total_tiles;      // elementwise tiles
   int32_t nmats;
-  int32_t xf_slot;          // which fp32 iterate buffer holds O'
+  int32_t xf_slot;          // which iterate buffer holds O' (fp32, or the bf16 high part)
+  int32_t split;            // bf16 mode: O' = high + low parts
   int32_t sumsq_per_tile;
   int32_t apply_kind;       // tile table the sums were recorded on
+  int32_t scale_mode;       // muon_scale_mode_t of the update
   float lr, wd, gamma;
+  float* diag;              // optional: diag[2 caller + 1] = RMS of the applied update O
 };
 
 // error bits in the device error word

@@ -16,7 +16,7 @@
 //                  ("Ch 06 · Muon" §3 and §5 Algorithm 1, regrouped), with
 //                  tcgen05.mma kind::f16, M = N = 128, K = 128 (zero padded).
 //
-// The elementwise kernel has already written the unscaled N (fp32 and bf16)
+// The elementwise kernel has already written the unscaled N (bf16 high and low parts)
 // and the normalisation scale s; step one folds s^2 into A and s into X'.
 // After the last step the update W <- W (1 - lr wd) - lr gamma sqrt(max(n, m))
 // O' goes to the caller's matrix in its orientation ("Muon 优化器完全拆解…",
@@ -140,11 +140,14 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       ptx::tma_load_3d(Xs, tm, bar_ld, 0, 0, md.index);
       ptx::tma_load_3d(Xs + kChunkBytes, tm, bar_ld, 64, 0, md.index);
     }
-    // fp32 iterate row `tid` into registers (zero outside the matrix)
+    // iterate row `tid` into fp32 registers, high + low bf16 parts (zero outside the matrix)
     float x[kS];
-    const float* xf = reinterpret_cast<const float*>(a.ws + gd.xf_off[0]) + (static_cast<int64_t>(md.index) * r + tid) * ldc;
+    const int64_t row_off = (static_cast<int64_t>(md.index) * r + tid) * ldc;
+    const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xb_off[0]) + row_off;
+    const __nv_bfloat16* xl = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xlo_off) + row_off;
 #pragma unroll
-    for (int e = 0; e < kS; ++e) x[e] = (tid < r && e < c) ? xf[e] : 0.f;
+    for (int e = 0; e < kS; ++e)
+      x[e] = (tid < r && e < c) ? __bfloat162float(xh[e]) + __bfloat162float(xl[e]) : 0.f;
     if (!ptx::mbar_wait(bar_ld, ld_phase, limit, abort_flag)) {
       *abort_flag = 1;
       atomicOr(a.err, kErrTimeout);
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
     float* T = reinterpret_cast<float*>(As);
 #pragma unroll
     for (int e = 0; e < kS; ++e) T[tid * kS + (e ^ (tid & 31))] = x[e];
-    if (a.scale_mode == kScaleUnitRms) {
+    if (a.scale_mode == kScaleUnitRms || a.diag) {
       // RMS(O') over the matrix (zeros outside it), in a fixed order
       float ssq = 0.f;
 #pragma unroll
@@ -248,10 +251,17 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       // unit-RMS: O = O' gamma / RMS(O'), a plain scale once RMS is known
       float gam = a.gamma;
       int mode = a.scale_mode;
+      const float rms = (mode == kScaleUnitRms || a.diag)
+                            ? sqrtf((red[0] + red[1] + red[2] + red[3]) / (static_cast<float>(r) * c))
+                            : 0.f;
       if (mode == kScaleUnitRms) {
-        const float rms = sqrtf((red[0] + red[1] + red[2] + red[3]) / (static_cast<float>(r) * c));
         gam = rms > 0.f ? a.gamma / rms : 0.f;
         mode = kScaleNone;
+      }
+      if (a.diag && tid == 0) {
+        // RMS of the applied update O = step / lr * O'
+        const UpdateConsts u1 = update_consts_raw(1.f, 0.f, gam, c, mode);
+        a.diag[2 * md.caller + 1] = u1.step * rms;
       }
       const UpdateConsts uc = update_consts_raw(a.lr, a.wd, gam, c, mode);
       const int lane = tid & 31;

@@ -10,7 +10,7 @@
 // two thirds of what a one-CTA 128 x 256 tile needs.
 //
 //   warp 0     TMA producer (both CTAs): 3-D tiled loads with 128-byte
-//              swizzle into a 4- or 5-deep ring; the bytes of both CTAs are
+//              swizzle into a 5- or 6-deep ring; the bytes of both CTAs are
 //              counted on the pair leader's mbarrier.
 //   warp 1     TMEM allocation (both CTAs); MMA issue (leader only):
 //              tcgen05.commit multicasts slot releases and finished
@@ -20,8 +20,16 @@
 //              reads 32 columns at a time from TMEM, stages results in
 //              swizzled shared memory and writes them with TMA tensor stores
 //              (whole lines, clipped at the matrix edge); inputs the
-//              epilogue needs (the fp32 iterate, the Gram tile, the weight)
+//              epilogue needs (the iterate, the Gram tile, the weight)
 //              arrive by double-buffered TMA loads.
+//
+// The iterate is stored as two bf16 parts, X = high + low: the high part is
+// the tensor-core operand (ping-pong, since every Apply tile reads the
+// current one), the low part, rn(X - high), is updated in place by the tile
+// that owns it. The pair carries 16 significant bits, enough for the a X term
+// (the same O' error as an fp32 iterate in a CPU emulation of the rounding),
+// and the Apply stage moves 4 bytes of iterate in and 4 out per element
+// instead of 4 + 4 + 2 with an fp32 master beside a bf16 operand copy.
 //
 // Stages ("Ch 06 · Muon" §3 and §5 Algorithm 1, regrouped as
 // a X + (b A + c A^2) X with A = X X^T):
@@ -31,9 +39,9 @@
 //              and, below the diagonal, mirrored. Step one folds s^2
 //              (X_0 = s N).
 //   Poly       B = b A + c A A^T (A symmetric), same tiling as Gram.
-//   Apply      X' = a X + B X: B is the K-major left operand, the iterate X
-//              the MN-major right operand (row-major X read as K x N). Step
-//              one folds s.
+//   Apply      X' = a X + B X: B is the K-major left operand, the iterate's
+//              high part the MN-major right operand (row-major X read as
+//              K x N); the epilogue adds a (high + low). Step one folds s.
 //   ApplyLast  the last step's Apply: O' = a X + B X, then the update of
 //              "Muon 优化器完全拆解…", Algorithm 1 steps four and five,
 //              W <- W (1 - lr wd) - lr gamma sqrt(max(n, m)) O', in the
@@ -68,21 +76,27 @@ constexpr int kEpiB16 = 32 * 32 * 2;              // bf16 32 x 32, 64-byte swizz
 constexpr size_t kBarrierBytes = 512;
 constexpr int kTmapBytes = 128;
 
-// Per-kind layout: ring depth and the epilogue staging slot (two per warp,
-// four epilogue warps, one per TMEM lane quarter):
-//   Gram       [bf16 out | bf16 mirror out]                       4 KB
-//   Poly       [bf16 A in | bf16 out | bf16 mirror out]           6 KB
-//   Apply      [fp32 iterate in / out | bf16 iterate out]         6 KB
-//   ApplyLast  [fp32 iterate in / O out | fp32 W in / out]        8 KB
+// Per-kind layout: ring depth and the epilogue staging slots (kEpiSlots per
+// warp, four epilogue warps, one per TMEM lane quarter). The Apply-like kinds
+// load an input per 32 x 32 chunk and keep kEpiSlots - 1 of those loads in
+// flight ahead of the chunk being processed; their epilogue, not the main
+// loop, sets the tile rate when the loads come from HBM. Slot sizes:
+//   Gram       [bf16 out | bf16 mirror out]                            4 KB
+//   Poly       [bf16 A in | bf16 out | bf16 mirror out]                6 KB
+//   Apply      [bf16 iterate high in / out | bf16 low in / out]        4 KB
+//   ApplyLast  [bf16 high in | bf16 low in, then fp32 O out | fp32 W in / out]  8 KB
+// The iterate is kept as two bf16 parts, X = high + low (16 significant
+// bits); the high part is the tensor-core operand.
 template <int KIND>
 struct Cfg {
   static constexpr int kEpiWarps = 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kStages = (KIND == kGram) ? 6 : (KIND == kApplyLast) ? 4 : 5;
   static constexpr int kSlot = (KIND == kApplyLast) ? 2 * kEpiF32
-                               : (KIND == kGram)    ? 2 * kEpiB16
-                                                    : kEpiF32 + kEpiB16;
-  static constexpr int kEpiBytes = kEpiWarps * 2 * kSlot;
+                               : (KIND == kPoly)    ? 3 * kEpiB16
+                                                    : 2 * kEpiB16;
+  static constexpr int kEpiSlots = (KIND == kApply) ? 4 : (KIND == kApplyLast) ? 3 : 2;
+  static constexpr int kEpiBytes = kEpiWarps * kEpiSlots * kSlot;
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarrierBytes;
   static constexpr bool kApplyLike = (KIND == kApply || KIND == kApplyLast);
   static constexpr int kTiles = kApplyLike ? kApply : KIND;  // which tile tables to walk
@@ -92,7 +106,7 @@ struct Cfg {
   static constexpr int kOffSymMirror = kOffSymOut + kEpiB16;
 };
 
-constexpr int kOffApplyOut16 = kEpiF32;
+constexpr int kOffLow = kEpiB16;   // low part of the iterate in Apply-like slots
 constexpr int kOffLastW = kEpiF32;
 
 constexpr uint32_t kIdescKK = ptx::idesc_bf16(kPairTile, kPairTile, 0, 0);   // both K-major
@@ -169,7 +183,7 @@ struct Smem {
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* drain;
-  uint64_t* eload;  // epilogue warps x 2
+  uint64_t* eload;  // epilogue warps x kEpiSlots
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -187,7 +201,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
   s.eload = s.drain + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + 2 * Cfg<KIND>::kEpiWarps);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + Cfg<KIND>::kEpiSlots * Cfg<KIND>::kEpiWarps);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
   return s;
 }
@@ -256,21 +270,27 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const GroupDes
   }
 }
 
-// X' (or O') = alpha (a X + acc) for one warp's 32 x 32 chunk; X from the
-// slot's fp32 input area.
+// X' (or O') = alpha (a X + acc) for one warp's 32 x 32 chunk; X = high +
+// low parts from the slot's two bf16 input areas.
 __device__ __forceinline__ void apply_values(const StageArgs& a, float alpha, const uint8_t* slot,
                                              const float (&v)[32], int lane, float (&x)[32]) {
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float4 p = *reinterpret_cast<const float4*>(slot + sw128_chunk(lane, q));
-    x[4 * q + 0] = alpha * fmaf(a.a, p.x, v[4 * q + 0]);
-    x[4 * q + 1] = alpha * fmaf(a.a, p.y, v[4 * q + 1]);
-    x[4 * q + 2] = alpha * fmaf(a.a, p.z, v[4 * q + 2]);
-    x[4 * q + 3] = alpha * fmaf(a.a, p.w, v[4 * q + 3]);
+  for (int q = 0; q < 4; ++q) {
+    const Bf16x8 h = *reinterpret_cast<const Bf16x8*>(slot + sw64_chunk(lane, q));
+    const Bf16x8 l = *reinterpret_cast<const Bf16x8*>(slot + kOffLow + sw64_chunk(lane, q));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 fh = __bfloat1622float2(h.v[k]);
+      const float2 fl = __bfloat1622float2(l.v[k]);
+      const int e = 8 * q + 2 * k;
+      x[e] = alpha * fmaf(a.a, fh.x + fl.x, v[e]);
+      x[e + 1] = alpha * fmaf(a.a, fh.y + fl.y, v[e + 1]);
+    }
   }
 }
 
-// Apply: write the new fp32 iterate and its bf16 operand copy.
+// Apply: write the new iterate as bf16 high part (the next operand) and low
+// part, high = rn(x'), low = rn(x' - high); x' - high is exact in fp32.
 // `ssq` accumulates this lane's sum of squares of the new iterate (used by
 // the unit-RMS update scale on the last step).
 __device__ __forceinline__ void epi_apply(const StageArgs& a, const GroupDesc& gd, const TileCoord& tc,
@@ -285,24 +305,26 @@ __device__ __forceinline__ void epi_apply(const StageArgs& a, const GroupDesc& g
 #pragma unroll
     for (int e = 0; e < 32; ++e) ssq = fmaf(x[e], x[e], ssq);
   }
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-    *reinterpret_cast<float4*>(slot + sw128_chunk(lane, q)) =
-        make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-  uint8_t* st16 = slot + kOffApplyOut16;
+  // each lane rewrites its own row of both areas: no other lane reads them
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    Bf16x8 p;
+    Bf16x8 h, l;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) p.v[h] = __floats2bfloat162_rn(x[8 * q + 2 * h], x[8 * q + 2 * h + 1]);
-    *reinterpret_cast<Bf16x8*>(st16 + sw64_chunk(lane, q)) = p;
+    for (int k = 0; k < 4; ++k) {
+      const int e = 8 * q + 2 * k;
+      h.v[k] = __floats2bfloat162_rn(x[e], x[e + 1]);
+      const float2 fh = __bfloat1622float2(h.v[k]);
+      l.v[k] = __floats2bfloat162_rn(x[e] - fh.x, x[e + 1] - fh.y);
+    }
+    *reinterpret_cast<Bf16x8*>(slot + sw64_chunk(lane, q)) = h;
+    *reinterpret_cast<Bf16x8*>(slot + kOffLow + sw64_chunk(lane, q)) = l;
   }
   ptx::fence_async_shared();
   __syncwarp();
   if (lane == 0) {
-    ptx::tma_store_3d(tmap(a, tc.g, kTmXfE), slot, col0, row0, static_cast<int>(tc.b));
-    ptx::tma_store_3d(tmap(a, tc.g, a.xsrc ? kTmXb0E : kTmXb1E), st16, col0, row0,
+    ptx::tma_store_3d(tmap(a, tc.g, a.xsrc ? kTmXb0E : kTmXb1E), slot, col0, row0,
                       static_cast<int>(tc.b));
+    ptx::tma_store_3d(tmap(a, tc.g, kTmXloE), slot + kOffLow, col0, row0, static_cast<int>(tc.b));
   }
 }
 
@@ -322,11 +344,16 @@ __device__ __forceinline__ void caller_xy(const MatDesc& md, int row0, int col0,
 // caller's orientation (transposed relative to the iterate when n > m).
 __device__ __forceinline__ void epi_apply_last(const StageArgs& a, const GroupDesc& gd,
                                                const TileCoord& tc, int row0, int col0, uint8_t* slot,
-                                               const float (&v)[32], int lane) {
+                                               const float (&v)[32], int lane, float& ssq) {
   const int mat = gd.first_mat + static_cast<int>(tc.b);
   const float alpha = a.first ? a.scale[mat] : 1.f;
   float x[32];
   apply_values(a, alpha, slot, v, lane, x);
+  if (a.sumsq_per_tile > 0) {
+    // update-RMS diagnostics; rows and columns past the matrix hold zeros
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ssq = fmaf(x[e], x[e], ssq);
+  }
   const MatDesc& md = a.mats[mat];
   const UpdateConsts uc = update_consts(a, gd.c);
   const bool tr = md.transposed != 0;
@@ -449,7 +476,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
       ptx::mbar_init(&s.tempty[i], 2 * kEpiWarps);
     }
     ptx::mbar_init(s.drain, 1);
-    for (int i = 0; i < 2 * kEpiWarps; ++i) ptx::mbar_init(&s.eload[i], 1);
+    for (int i = 0; i < C::kEpiSlots * kEpiWarps; ++i) ptx::mbar_init(&s.eload[i], 1);
     *s.abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -572,12 +599,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
     const int quarter = warp & 3;  // TMEM lanes this warp may read: 32 * quarter ...
     const int ch_begin = (ew / 4) * C::kChunksPerWarp;  // this warp's share of the columns
     const int ch_end = ch_begin + C::kChunksPerWarp;
-    uint8_t* slots = s.epi + ew * 2 * C::kSlot;
-    uint64_t* eload = s.eload + 2 * ew;
-    uint32_t eload_phase[2] = {0u, 0u};
+    constexpr int S = C::kEpiSlots;
+    uint8_t* slots = s.epi + ew * S * C::kSlot;
+    uint64_t* eload = s.eload + S * ew;
+    uint32_t eload_phase = 0u;  // bit i: phase of slot i's load barrier
     uint32_t leader_tempty[2];
     for (int i = 0; i < 2; ++i) leader_tempty[i] = ptx::mapa_shared(ptx::smem_u32(&s.tempty[i]), 0);
     constexpr bool kInput = (KIND != kGram);
+    // input loads in flight ahead of the current chunk: with three or more
+    // slots the newest chunk's stores may still be reading their slot when the
+    // next load is issued (no wait on them); with two they must have finished
+    constexpr int D = !kInput ? 0 : (S >= 3 ? S - 2 : S - 1);
+    constexpr int kReuseWait = S - 1 - D;  // store groups that may still be pending
     uint32_t acc = 0, acc_phase = 0;
     bool ok = true;
     for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
@@ -587,7 +620,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
       const int bi = (tc.I * kPairTile + static_cast<int>(rank) * kHalf) / kHalf;
       const int bz = static_cast<int>(tc.b);
       const int mat = gd.first_mat + bz;
-      const void* in_map = tmap(a, tc.g, C::kApplyLike ? kTmXfE : kTmAE);
+      // Apply-like: the current iterate's high part (the operand buffer) and low part
+      const void* in_map = tmap(a, tc.g, C::kApplyLike ? (a.xsrc ? kTmXb1E : kTmXb0E) : kTmAE);
       float ssq = 0.f;  // sum of squares of this warp's share of X' (unit-RMS scale)
       // the last step also brings the weight chunk, in the caller's orientation
       bool w_in = false;
@@ -601,66 +635,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
           if (md.O) ptx::fence_tmap_acquire(mat_tmap(a, mat, kMtO));
         }
       }
-      const uint32_t in_bytes = (KIND == kPoly ? kEpiB16 : kEpiF32) + (w_in ? kEpiF32 : 0);
-      auto issue_load = [&](int ch) {
-        // the slot's previous stores must have finished reading it
-        ptx::bulk_wait_read<0>();
-        uint8_t* slot = slots + (ch & 1) * C::kSlot;
-        uint64_t* bar = &eload[ch & 1];
+      const uint32_t in_bytes = (KIND == kPoly ? kEpiB16 : 2 * kEpiB16) + (w_in ? kEpiF32 : 0);
+      const int limit_c = C::kApplyLike ? gd.c : gd.r;
+      // rows or columns past the matrix: nothing to load or store for a chunk
+      auto live_chunk = [&](int ch) {
+        return ch < ch_end && row0 < gd.r && tc.J * kPairTile + ch * 32 < limit_c;
+      };
+      auto issue_load = [&](int ch) {  // the caller has made sure the slot is free
+        const int sl = (ch - ch_begin) % S;
+        uint8_t* slot = slots + sl * C::kSlot;
+        uint64_t* bar = &eload[sl];
         const int col0 = tc.J * kPairTile + ch * 32;
         ptx::mbar_arrive_expect_tx(bar, in_bytes);
         ptx::tma_load_3d(slot, in_map, bar, col0, row0, bz);
+        if (C::kApplyLike) ptx::tma_load_3d(slot + kOffLow, tmap(a, tc.g, kTmXloE), bar, col0, row0, bz);
         if (KIND == kApplyLast && w_in)
           ptx::tma_load_3d(slot + kOffLastW, mat_tmap(a, mat, kMtW), bar, w_tr ? row0 : col0,
                            w_tr ? col0 : row0, 0);
       };
-      if (kInput && lane == 0 && row0 < gd.r && tc.J * kPairTile + ch_begin * 32 < (C::kApplyLike ? gd.c : gd.r))
-        issue_load(ch_begin);
+      if (kInput && lane == 0) {
+        ptx::bulk_wait_read<0>();  // the previous tile's stores have read every slot
+        for (int ch = ch_begin; ch < ch_begin + D; ++ch)
+          if (live_chunk(ch)) issue_load(ch);
+      }
       if (!ptx::mbar_wait(&s.tfull[acc], acc_phase, limit, s.abort_flag)) {
         raise_abort(a, s);
         ok = false;
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
-      const int limit_c = C::kApplyLike ? gd.c : gd.r;
 #pragma unroll 1
       for (int ch = ch_begin; ok && ch < ch_end; ++ch) {
-        uint8_t* slot = slots + (ch & 1) * C::kSlot;
+        const int sl = (ch - ch_begin) % S;
+        uint8_t* slot = slots + sl * C::kSlot;
         const int col0 = tc.J * kPairTile + ch * 32;
-        // rows or columns past the matrix: nothing to load or store for this chunk
-        const bool live = row0 < gd.r && col0 < limit_c;
-        const bool next_live = row0 < gd.r && col0 + 32 < limit_c && ch + 1 < ch_end;
+        const bool live = live_chunk(ch);
         if (lane == 0) {
-          if (kInput && next_live) issue_load(ch + 1);
-          if (!kInput) ptx::bulk_wait_read<1>();
+          // the load D chunks ahead reuses the slot of chunk ch + D - S, whose
+          // stores are older than the newest kReuseWait groups
+          if (kInput && live_chunk(ch + D)) {
+            ptx::bulk_wait_read<kReuseWait>();
+            issue_load(ch + D);
+          }
+          if (!kInput) ptx::bulk_wait_read<1>();  // two slots: chunk ch - 2's stores have read it
         }
         __syncwarp();
         float v[32];
         ptx::tmem_ld32(taddr + ch * 32, v);
         if (kInput && live) {
-          if (!ptx::mbar_wait(&eload[ch & 1], eload_phase[ch & 1], limit, s.abort_flag)) {
+          if (!ptx::mbar_wait(&eload[sl], (eload_phase >> sl) & 1u, limit, s.abort_flag)) {
             raise_abort(a, s);
             ok = false;
             break;
           }
-          eload_phase[ch & 1] ^= 1u;
+          eload_phase ^= 1u << sl;
         }
         if (live) {
           if (KIND == kApply) {
             epi_apply(a, gd, tc, row0, col0, slot, v, lane, ssq);
           } else if (KIND == kApplyLast) {
-            epi_apply_last(a, gd, tc, row0, col0, slot, v, lane);
+            epi_apply_last(a, gd, tc, row0, col0, slot, v, lane, ssq);
           } else {
             const int bj = col0 / kHalf;
             if (bj <= bi) epi_symmetric<KIND>(a, gd, tc, row0, col0, bj < bi, slot, v, lane);
           }
         }
         // one bulk group per chunk (possibly empty), so "all but the newest
-        // group" always means "the chunk that used the other slot"
+        // group" always means "every chunk before the previous one"
         __syncwarp();
         if (lane == 0) ptx::bulk_commit();
       }
-      if (KIND == kApply && a.sumsq_per_tile > 0) {
+      if ((KIND == kApply || KIND == kApplyLast) && a.sumsq_per_tile > 0) {
         // one slot per (tile, CTA of the pair, epilogue warp); every slot is written
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);

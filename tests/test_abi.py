@@ -15,7 +15,8 @@ from muon_step_b200._lib import (MUON_ERR_INVALID_ARG, MUON_ERR_WORKSPACE, MUON_
                                  MuonParam)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "muon_step.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -26,7 +27,7 @@ def lib():
 
 
 def header_symbols():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"^MUON_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)))
 
 
@@ -126,8 +127,8 @@ def expected_workspace(shapes, prec):
     al = lambda x, a: (x + a - 1) // a * a
     ng, nm = len(groups), len(shapes)
     ew = sum(math.ceil(n / 32) * math.ceil(m / 128) for n, m in shapes)
-    off = al(ng * 152, 256)          # GroupDesc is 152 bytes
-    off = al(off + nm * 80, 256)     # MatDesc is 80 bytes
+    off = al(ng * 160, 256)          # GroupDesc is 160 bytes
+    off = al(off + nm * 88, 256)     # MatDesc is 88 bytes
     off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + ew * 4, 256)     # matrix of each elementwise tile
@@ -152,7 +153,8 @@ def expected_workspace(shapes, prec):
         x = k * r * al(c, 8)
         a = k * r * al(r, 8)
         if prec == MUON_NS_BF16:
-            for nbytes in (4 * x, 2 * x, 2 * x, 2 * a, 2 * a):
+            # iterate high part (two, ping-pong) and low part, bf16; A; B
+            for nbytes in (2 * x, 2 * x, 2 * x, 2 * a, 2 * a):
                 off = al(off + nbytes, 1024)
         else:
             for nbytes in (4 * x, 4 * x, 4 * a, 4 * a):
@@ -220,11 +222,24 @@ def test_scale_modes_change_the_launch_list(lib):
     assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
     assert kinds_now() == [0, 5]
     lib.muon_plan_destroy(plan)
+    # diagnostics add one reduction after the fused last step (shape / none scale)
+    st, plan = create(lib, [(64, 64), (300, 400)])
+    shape = kinds_now()
+    assert lib.muon_plan_set_diagnostics(plan, ctypes.c_void_p(FAKE)) == MUON_OK
+    assert kinds_now() == shape + [6]
+    assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
+    assert kinds_now() == shape[:-1] + [3, 6, 7]
+    assert lib.muon_plan_set_diagnostics(plan, None) == MUON_OK
+    assert lib.muon_plan_set_scale_mode(plan, 0) == MUON_OK
+    assert kinds_now() == shape
+    assert lib.muon_plan_set_diagnostics(plan, ctypes.c_void_p(FAKE + 2)) == MUON_ERR_INVALID_ARG
+    lib.muon_plan_destroy(plan)
     # orthogonalisation plans have no update to scale
     ns = ctypes.c_void_p()
     mats = (MuonNsMatrix * 1)(MuonNsMatrix(FAKE, 2 * FAKE, 5, 9))
     assert lib.muon_plan_create_ns(mats, 1, MUON_NS_BF16, None, ctypes.byref(ns)) == MUON_OK
     assert lib.muon_plan_set_scale_mode(ns, 1) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_set_diagnostics(ns, ctypes.c_void_p(FAKE)) == MUON_ERR_INVALID_ARG
     lib.muon_plan_destroy(ns)
 
 

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import workloads
-from tests.parity import TOL_ELEMENTWISE, TOL_O, all_within, check_ns, check_step, rel
+from tests.parity import TOL_ELEMENTWISE, TOL_O, all_within, check_ns, check_step, rel, tol_o
 
 pytestmark = pytest.mark.gpu
 
@@ -206,3 +206,48 @@ def test_scale_modes(precision, scale_mode):
     worst = check_step(wl, precision, hyper=hyper, scale_mode=scale_mode)
     assert worst["O_over_tol"] <= 1.0, worst
     assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("scale_mode", ["shape", "unit_rms", "none"])
+def test_diagnostics(precision, scale_mode):
+    """||N||_F and RMS(O) per matrix, in the caller's order, against the
+    oracle: the norm to fp32 rounding of a double sum; the update RMS against
+    the RMS of the GPU's own O' to 1e-5 (the epilogue sums in fp32), and
+    against the full oracle within the O' tolerance."""
+    import muon_step_b200 as ms
+    from oracle import companion_oracle
+
+    shapes = [(300, 520), (64, 64), (520, 300), (1, 7), (257, 129), (100, 37)]
+    wl = workloads.make_random(shapes, device="cuda", seed=31)
+    h = wl.hyper
+    before = [(wl.G[k].double().cpu().numpy(), wl.M[k].double().cpu().numpy())
+              for k in range(wl.count)]
+    O = [torch.empty_like(wl.W[k]) for k in range(wl.count)]
+    plan = ms.MuonPlan([(wl.W[k], wl.G[k], wl.M[k], O[k]) for k in range(wl.count)],
+                       precision=precision, scale_mode=scale_mode)
+    diag = torch.full((wl.count, 2), -1.0, device="cuda")
+    plan.set_diagnostics(diag)
+    ws = plan.alloc_workspace()
+    plan.execute(ws, lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"], gamma=h["gamma"],
+                 nesterov=h["nesterov"])
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    got = diag.double().cpu().numpy()
+    for k in range(wl.count):
+        G, Mp = before[k]
+        n, m = G.shape
+        norm, rms_o = companion_oracle.muon_step_diagnostics(
+            G, Mp, n, m, mu=h["mu"], gamma=h["gamma"], nesterov_on=h["nesterov"],
+            scale_mode=scale_mode)
+        assert abs(got[k, 0] - norm) <= 1e-6 * norm, (k, got[k, 0], norm)
+        Og = O[k].double().cpu().numpy()
+        r = companion_oracle.rms(Og)
+        if scale_mode == "shape":
+            own = h["gamma"] * math.sqrt(max(n, m)) * r
+        elif scale_mode == "unit_rms":
+            own = h["gamma"] if r > 0 else 0.0
+        else:
+            own = h["gamma"] * r
+        assert abs(got[k, 1] - own) <= 1e-5 * own, (k, got[k, 1], own)
+        assert abs(got[k, 1] - rms_o) <= tol_o(precision, (n, m)) * rms_o, (k, got[k, 1], rms_o)
