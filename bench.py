@@ -213,6 +213,8 @@ def time_adamw_companion(wl, steps, dev, stream, peaks, world):
     and a prediction head of ADAMW_VOCAB rows by the model width (the most
     common matrix dimension), plus two norm vectors per matrix. One launch per
     step, timed with CUDA events over `steps` steps; HBM-bound, 28 B/element."""
+    import torch
+
     import muon_step_b200 as ms
 
     dims = {}
