@@ -35,6 +35,7 @@ EXPORTS = (
     "muon_adamw_plan_create", "muon_adamw_plan_workspace_size", "muon_adamw_plan_execute",
     "muon_adamw_plan_numel", "muon_adamw_plan_destroy", "muon_adamw_workspace_size",
     "muon_adamw_step",
+    "muon_shard_workspace_size", "muon_shard_momentum", "muon_shard_update",
 )
 
 
@@ -62,6 +63,16 @@ class AdamwHyper(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("step", ctypes.c_int32), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
                 ("step_dev", ctypes.c_void_p)]
+
+
+class ShardMomentum(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_void_p), ("G", ctypes.c_void_p), ("N", ctypes.c_void_p),
+                ("numel", ctypes.c_int64)]
+
+
+class ShardUpdate(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("O", ctypes.c_void_p), ("numel", ctypes.c_int64),
+                ("n", ctypes.c_int64), ("m", ctypes.c_int64)]
 
 
 class MuonHyper(ctypes.Structure):
@@ -104,6 +115,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_adamw_workspace_size": (st, [P(AdamwParam), ctypes.c_int, P(ctypes.c_size_t)]),
         "muon_adamw_step": (st, [P(AdamwParam), ctypes.c_int, P(AdamwHyper), vp, ctypes.c_size_t,
                                  vp]),
+        "muon_shard_workspace_size": (st, [ctypes.c_int, P(ctypes.c_size_t)]),
+        "muon_shard_momentum": (st, [P(ShardMomentum), ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                     vp, ctypes.c_size_t, vp]),
+        "muon_shard_update": (st, [P(ShardUpdate), ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                   ctypes.c_float, vp, ctypes.c_size_t, vp]),
         "muon_workspace_size": (st, [P(MuonParam), ctypes.c_int, ctypes.c_int, P(ctypes.c_size_t)]),
         "muon_step": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                            ctypes.c_float, ctypes.c_int, P(MuonNsSchedule), ctypes.c_int, vp,

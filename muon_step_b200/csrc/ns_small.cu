@@ -145,9 +145,26 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
     const int64_t row_off = (static_cast<int64_t>(md.index) * r + tid) * ldc;
     const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xb_off[0]) + row_off;
     const __nv_bfloat16* xl = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xlo_off) + row_off;
+    // 16-byte loads: rows start 16-byte aligned (ldc is a multiple of 8) and
+    // the 8-element groups that start below c lie inside the row's ldc
 #pragma unroll
-    for (int e = 0; e < kS; ++e)
-      x[e] = (tid < r && e < c) ? __bfloat162float(xh[e]) + __bfloat162float(xl[e]) : 0.f;
+    for (int q = 0; q < kS / 8; ++q) {
+      uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;
+      if (tid < r && 8 * q < c) {
+        hv = *reinterpret_cast<const uint4*>(xh + 8 * q);
+        lv = *reinterpret_cast<const uint4*>(xl + 8 * q);
+      }
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hv);
+      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lv);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 fh = __bfloat1622float2(h2[k]);
+        const float2 fl = __bfloat1622float2(l2[k]);
+        const int e = 8 * q + 2 * k;
+        x[e] = e < c ? fh.x + fl.x : 0.f;  // columns c .. ldc of the buffers are not written
+        x[e + 1] = e + 1 < c ? fh.y + fl.y : 0.f;
+      }
+    }
     if (!ptx::mbar_wait(bar_ld, ld_phase, limit, abort_flag)) {
       *abort_flag = 1;
       atomicOr(a.err, kErrTimeout);

@@ -1,0 +1,212 @@
+// Elementwise steps of the ZeRO-sharded Muon step over lists of shards.
+//
+// [V4-breakdown] "Muon 优化器完全拆解…", section "分布式工程", Algorithm 1
+// "Distributed Muon": the momentum update on the local gradient shard (step 2)
+// and the parameter update with the local shard of the orthogonalised matrix
+// (step 6). The arithmetic repeats that of the single-GPU step exactly:
+// M = fma(mu, M, G), N = fma(mu, M, G) as in the elementwise front kernel,
+// W = fma(W, 1 - lr wd, -(lr gamma sqrt(c)) O) as in the last Apply epilogue.
+//
+// Layout as in the AdamW kernel: shards cut into 4096-element chunks, one CTA
+// of 256 threads per chunk, 16-byte accesses when every pointer of the shard
+// is 16-byte aligned, all loads of a thread before its first store.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "muon_shard.h"
+#include "stage_common.cuh"
+
+namespace muon {
+
+muon_status_t current_device_checked(int* dev);
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kGroups = 4;
+constexpr int64_t kChunk = kThreads * 4 * kGroups;
+constexpr int64_t kMaxNumel = int64_t(1) << 40;
+
+struct ShardItem {
+  float* a;           // M (momentum) or W (update), in place
+  const float* b;     // G or O
+  float* c;           // N (momentum) or unused
+  int64_t numel;
+  int64_t chunk_begin;
+  int32_t vec;
+  int32_t cdim;       // update: max(n, m) of the whole matrix
+};
+
+struct ShardArgs {
+  const ShardItem* items;
+  int32_t count;
+  int32_t nesterov;
+  float mu;
+  float lr, wd, gamma;
+};
+
+template <bool kMomentum>
+__device__ __forceinline__ void elem(const ShardArgs& s, const UpdateConsts& uc, float& a, float b,
+                                     float& c) {
+  if (kMomentum) {
+    a = fmaf(s.mu, a, b);
+    c = s.nesterov ? fmaf(s.mu, a, b) : a;
+  } else {
+    a = fmaf(a, uc.keep, -uc.step * b);
+  }
+}
+
+template <bool kMomentum>
+__global__ void __launch_bounds__(kThreads) shard_kernel(const __grid_constant__ ShardArgs s) {
+  __shared__ int item_s;
+  const int64_t chunk = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int lo = 0, hi = s.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(&s.items[mid].chunk_begin) <= chunk) lo = mid;
+      else hi = mid - 1;
+    }
+    item_s = lo;
+  }
+  __syncthreads();
+  const ShardItem it = s.items[item_s];
+  const UpdateConsts uc = update_consts_raw(s.lr, s.wd, s.gamma, kMomentum ? 1 : it.cdim);
+  const int64_t base = (chunk - it.chunk_begin) * kChunk;
+  const int tid = threadIdx.x;
+  if (it.vec && base + kChunk <= it.numel) {
+    float4 a[kGroups], b[kGroups], c[kGroups];
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      const int64_t i = base + q * (kThreads * 4) + tid * 4;
+      a[q] = *reinterpret_cast<const float4*>(it.a + i);
+      b[q] = __ldcs(reinterpret_cast<const float4*>(it.b + i));
+    }
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      elem<kMomentum>(s, uc, a[q].x, b[q].x, c[q].x);
+      elem<kMomentum>(s, uc, a[q].y, b[q].y, c[q].y);
+      elem<kMomentum>(s, uc, a[q].z, b[q].z, c[q].z);
+      elem<kMomentum>(s, uc, a[q].w, b[q].w, c[q].w);
+    }
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      const int64_t i = base + q * (kThreads * 4) + tid * 4;
+      *reinterpret_cast<float4*>(it.a + i) = a[q];
+      if (kMomentum) *reinterpret_cast<float4*>(it.c + i) = c[q];
+    }
+  } else {
+    for (int e = tid; e < kChunk; e += kThreads) {
+      const int64_t i = base + e;
+      if (i >= it.numel) break;
+      float a = it.a[i], c = 0.f;
+      elem<kMomentum>(s, uc, a, it.b[i], c);
+      it.a[i] = a;
+      if (kMomentum) it.c[i] = c;
+    }
+  }
+}
+
+size_t table_bytes(int count) {
+  return (static_cast<size_t>(std::max(count, 1)) * sizeof(ShardItem) + 255) / 256 * 256;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+template <bool kMomentum>
+muon_status_t launch(std::vector<ShardItem>& items, int64_t chunks, ShardArgs args, void* workspace,
+                     size_t workspace_bytes, void* stream_ptr) {
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < table_bytes(static_cast<int>(items.size())))
+    return MUON_ERR_WORKSPACE;
+  int dev = 0;
+  muon_status_t st = current_device_checked(&dev);
+  if (st != MUON_OK) return st;
+  if (chunks == 0) return MUON_OK;
+  if (chunks > 0x7fffffffLL) return MUON_ERR_UNSUPPORTED;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (cudaMemcpyAsync(workspace, items.data(), items.size() * sizeof(ShardItem),
+                      cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  args.items = static_cast<const ShardItem*>(workspace);
+  args.count = static_cast<int32_t>(items.size());
+  shard_kernel<kMomentum><<<static_cast<unsigned>(chunks), kThreads, 0, stream>>>(args);
+  return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace muon
+
+extern "C" {
+
+muon_status_t muon_shard_workspace_size(int count, size_t* bytes) {
+  if (!bytes || count < 1) return MUON_ERR_INVALID_ARG;
+  *bytes = muon::table_bytes(count);
+  return MUON_OK;
+}
+
+muon_status_t muon_shard_momentum(const muon_shard_momentum_t* shards, int count, float momentum,
+                                  int nesterov, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  using namespace muon;
+  if (!shards || count < 1 || !std::isfinite(momentum)) return MUON_ERR_INVALID_ARG;
+  std::vector<ShardItem> items;
+  int64_t chunks = 0;
+  for (int k = 0; k < count; ++k) {
+    const muon_shard_momentum_t& q = shards[k];
+    if (q.numel < 0 || q.numel > kMaxNumel) return MUON_ERR_INVALID_ARG;
+    if (q.numel == 0) continue;
+    if (!q.M || !q.G || !q.N || !aligned(q.M, 4) || !aligned(q.G, 4) || !aligned(q.N, 4))
+      return MUON_ERR_INVALID_ARG;
+    ShardItem it{};
+    it.a = q.M;
+    it.b = q.G;
+    it.c = q.N;
+    it.numel = q.numel;
+    it.chunk_begin = chunks;
+    it.vec = aligned(q.M, 16) && aligned(q.G, 16) && aligned(q.N, 16);
+    chunks += (q.numel + kChunk - 1) / kChunk;
+    items.push_back(it);
+  }
+  ShardArgs a{};
+  a.mu = momentum;
+  a.nesterov = nesterov ? 1 : 0;
+  return launch<true>(items, chunks, a, workspace, workspace_bytes, stream);
+}
+
+muon_status_t muon_shard_update(const muon_shard_update_t* shards, int count, float lr,
+                                float weight_decay, float gamma, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  using namespace muon;
+  if (!shards || count < 1 || !std::isfinite(lr) || !std::isfinite(weight_decay) ||
+      !std::isfinite(gamma))
+    return MUON_ERR_INVALID_ARG;
+  std::vector<ShardItem> items;
+  int64_t chunks = 0;
+  for (int k = 0; k < count; ++k) {
+    const muon_shard_update_t& q = shards[k];
+    if (q.numel < 0 || q.numel > kMaxNumel || q.n < 1 || q.m < 1 || q.n > 0x7fffffffLL ||
+        q.m > 0x7fffffffLL)
+      return MUON_ERR_INVALID_ARG;
+    if (q.numel == 0) continue;
+    if (!q.W || !q.O || !aligned(q.W, 4) || !aligned(q.O, 4)) return MUON_ERR_INVALID_ARG;
+    ShardItem it{};
+    it.a = q.W;
+    it.b = q.O;
+    it.numel = q.numel;
+    it.chunk_begin = chunks;
+    it.vec = aligned(q.W, 16) && aligned(q.O, 16);
+    it.cdim = static_cast<int32_t>(std::max(q.n, q.m));
+    chunks += (q.numel + kChunk - 1) / kChunk;
+    items.push_back(it);
+  }
+  ShardArgs a{};
+  a.lr = lr;
+  a.wd = weight_decay;
+  a.gamma = gamma;
+  return launch<false>(items, chunks, a, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"

@@ -19,6 +19,7 @@ One process per GPU, torch.distributed for the plumbing.
 
 from __future__ import annotations
 
+import ctypes
 from typing import Callable, Optional, Sequence
 
 import torch
@@ -112,3 +113,146 @@ class DistributedMuon:
                 W = self.params[k][0]
                 W.copy_(self._bufs[r][off:off + W.numel()].view_as(W))
                 off += W.numel()
+
+
+# ---------------------------------------------------------------------------
+# ZeRO-sharded Distributed Muon
+# ---------------------------------------------------------------------------
+
+def shard_size(numel: int, world: int) -> int:
+    """Elements of one rank's shard of a flattened matrix: the matrix is
+    padded to world equal shards, each a multiple of 4 elements (16 bytes)."""
+    per = -(-numel // world)
+    return -(-per // 4) * 4
+
+
+class _ShardKernels:
+    """The library's shard kernels and ns_orthogonalize (C ABI)."""
+
+    def __init__(self, n_items, device):
+        from . import _lib
+        self._lib = _lib.load()
+        nbytes = ctypes.c_size_t()
+        st = self._lib.muon_shard_workspace_size(n_items, ctypes.byref(nbytes))
+        if st != 0:
+            raise RuntimeError(f"muon_shard_workspace_size: status {st}")
+        self.ws = torch.empty(max(nbytes.value, 256), dtype=torch.uint8, device=device)
+        self.ns_plan = None
+        self.ns_ws = None
+
+    def _stream(self):
+        return torch.cuda.current_stream().cuda_stream
+
+    def momentum(self, items, mu, nesterov):
+        from ._lib import ShardMomentum
+        arr = (ShardMomentum * len(items))(*[ShardMomentum(M.data_ptr(), G.data_ptr(), N.data_ptr(),
+                                                           M.numel()) for M, G, N in items])
+        st = self._lib.muon_shard_momentum(arr, len(items), mu, 1 if nesterov else 0,
+                                           self.ws.data_ptr(), self.ws.numel(), self._stream())
+        if st != 0:
+            raise RuntimeError(f"muon_shard_momentum: status {st}")
+
+    def orthogonalize(self, pairs, precision, schedule, eps):
+        from . import NsPlan
+        if self.ns_plan is None:
+            self.ns_plan = NsPlan(pairs, precision=precision, schedule=schedule, eps=eps)
+            self.ns_ws = self.ns_plan.alloc_workspace()
+        self.ns_plan.execute(self.ns_ws)
+
+    def update(self, items, lr, wd, gamma):
+        from ._lib import ShardUpdate
+        arr = (ShardUpdate * len(items))(*[ShardUpdate(W.data_ptr(), O.data_ptr(), W.numel(), n, m)
+                                           for W, O, (n, m) in items])
+        st = self._lib.muon_shard_update(arr, len(items), lr, wd, gamma, self.ws.data_ptr(),
+                                         self.ws.numel(), self._stream())
+        if st != 0:
+            raise RuntimeError(f"muon_shard_update: status {st}")
+
+
+class ZeroMuon:
+    """Distributed Muon with momentum and weights sharded over the ranks of
+    ``group`` ([V4-breakdown] section "分布式工程", Algorithm 1 "Distributed
+    Muon"). Each matrix is flattened and padded to ``world`` equal shards; rank
+    r keeps shard r of the momentum. One step:
+
+      1. reduce-scatter (sum) of every rank's local gradient -> gradient shard
+      2. momentum + Nesterov on the shard (library kernel, one launch)
+      3. all-gather of the Nesterov shards -> the whole N on every rank
+      4. Newton-Schulz on the whole matrices (library ns_orthogonalize)
+      5./6. decay + update of this rank's weight shard with its shard of O'
+         (library kernel, one launch)
+      7. all-gather of the weight shards -> the whole updated weights
+
+    Every rank computes the Newton-Schulz of every matrix, as the algorithm
+    states (the whole matrix is gathered everywhere). Weights, gradients and
+    the gathered buffers are owned here, flat and padded; ``weight(k)`` and
+    ``grad(k)`` are their n x m views. Write each step's local gradient into
+    ``grad(k)`` (scaled as the caller wants the sum over ranks to be).
+    ``kernels`` replaces the library calls (tests on CPU ranks).
+    """
+
+    def __init__(self, shapes: Sequence, group=None, device=None, precision="bf16",
+                 schedule=None, eps=None, kernels=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.shapes = [tuple(int(d) for d in s) for s in shapes]
+        if not self.shapes or any(len(s) != 2 for s in self.shapes):
+            raise ValueError("ZeroMuon takes a non-empty list of 2-D shapes")
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.precision, self.schedule, self.eps = precision, schedule, eps
+        self.shard = [shard_size(n * m, self.world) for n, m in self.shapes]
+        full = [s * self.world for s in self.shard]
+        z = lambda k: torch.zeros(k, dtype=torch.float32, device=dev)
+        self._W = [z(f) for f in full]        # whole weights (padded); shard r is this rank's
+        self._G = [z(f) for f in full]        # local gradient (padded)
+        self._N = [z(f) for f in full]        # gathered Nesterov input (padded)
+        self._O = [z(f) for f in full]        # O' of the whole matrix (padded)
+        self.momentum_shards = [z(s) for s in self.shard]
+        self._g = [z(s) for s in self.shard]  # reduced gradient shard
+        self.kernels = kernels if kernels is not None else _ShardKernels(len(self.shapes), dev)
+        self._in_place = dist.get_backend(group) == "nccl"
+
+    def _view(self, buf, k):
+        n, m = self.shapes[k]
+        return buf[k][: n * m].view(n, m)
+
+    def _mine(self, buf, k):
+        s = self.shard[k]
+        return buf[k][self.rank * s:(self.rank + 1) * s]
+
+    def weight(self, k):
+        return self._view(self._W, k)
+
+    def grad(self, k):
+        return self._view(self._G, k)
+
+    def load_weights(self, weights):
+        """Copy the initial whole weights (identical on every rank)."""
+        for k, W in enumerate(weights):
+            self.weight(k).copy_(W)
+
+    def step(self, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True):
+        K = len(self.shapes)
+        for k in range(K):  # 1. gradient shards
+            dist.reduce_scatter_tensor(self._g[k], self._G[k], group=self.group)
+        # 2. momentum on the shards, Nesterov shard written into its slot of N
+        self.kernels.momentum([(self.momentum_shards[k], self._g[k], self._mine(self._N, k))
+                               for k in range(K)], momentum, nesterov)
+        for k in range(K):  # 3. whole N on every rank
+            dist.all_gather_into_tensor(self._N[k], self._gather_src(self._N, k), group=self.group)
+        # 4. Newton-Schulz of every whole matrix
+        self.kernels.orthogonalize([(self._view(self._N, k), self._view(self._O, k)) for k in range(K)],
+                                   self.precision, self.schedule, self.eps)
+        # 5./6. update of this rank's weight shards
+        self.kernels.update([(self._mine(self._W, k), self._mine(self._O, k), self.shapes[k])
+                             for k in range(K)], lr, weight_decay, gamma)
+        for k in range(K):  # 7. whole updated weights
+            dist.all_gather_into_tensor(self._W[k], self._gather_src(self._W, k), group=self.group)
+
+    def _gather_src(self, buf, k):
+        # NCCL gathers in place (the input is the output's own slot); other
+        # backends get a copy of the slot
+        mine = self._mine(buf, k)
+        return mine if self._in_place else mine.clone()

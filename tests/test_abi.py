@@ -276,3 +276,28 @@ def test_timing_events_need_two_per_launch(lib):
     assert lib.muon_plan_set_events(plan, ev, 62) == MUON_OK
     assert lib.muon_plan_set_events(plan, None, 0) == MUON_OK
     lib.muon_plan_destroy(plan)
+
+
+def test_shard_calls_validate_before_touching_a_device(lib):
+    from muon_step_b200._lib import ShardMomentum, ShardUpdate
+    n = ctypes.c_size_t()
+    assert lib.muon_shard_workspace_size(0, ctypes.byref(n)) == MUON_ERR_INVALID_ARG
+    assert lib.muon_shard_workspace_size(5, ctypes.byref(n)) == MUON_OK and n.value == 256
+    assert lib.muon_shard_workspace_size(6, ctypes.byref(n)) == MUON_OK and n.value == 512  # 48 B each
+    ws = ctypes.c_void_p(1 << 20)
+    mom = (ShardMomentum * 1)(ShardMomentum(FAKE, FAKE + 4096, FAKE + 8192, -1))
+    assert lib.muon_shard_momentum(mom, 1, 0.95, 1, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    mom[0] = ShardMomentum(FAKE, None, FAKE + 8192, 16)
+    assert lib.muon_shard_momentum(mom, 1, 0.95, 1, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    mom[0] = ShardMomentum(FAKE + 2, FAKE + 4096, FAKE + 8192, 16)
+    assert lib.muon_shard_momentum(mom, 1, 0.95, 1, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    assert lib.muon_shard_momentum(mom, 0, 0.95, 1, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    mom[0] = ShardMomentum(FAKE, FAKE + 4096, FAKE + 8192, 16)
+    assert lib.muon_shard_momentum(mom, 1, float("nan"), 1, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    assert lib.muon_shard_momentum(mom, 1, 0.95, 1, ctypes.c_void_p((1 << 20) + 8), 1 << 20,
+                                   None) == MUON_ERR_WORKSPACE
+    upd = (ShardUpdate * 1)(ShardUpdate(FAKE, FAKE + 4096, 16, 0, 4))
+    assert lib.muon_shard_update(upd, 1, 0.02, 0.1, 0.2, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    upd[0] = ShardUpdate(FAKE, FAKE + 4096, 16, 4, 4)
+    assert lib.muon_shard_update(upd, 1, float("inf"), 0.1, 0.2, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
+    assert lib.muon_shard_update(upd, 1, 0.02, 0.1, 0.2, ws, 16, None) == MUON_ERR_WORKSPACE

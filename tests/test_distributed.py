@@ -133,3 +133,84 @@ def test_distributed_step_matches_single_process(tmp_path, world):
                 assert torch.equal(out["M"][k], ref[k][2])
             else:
                 assert torch.equal(out["M"][k], _inputs()[k][2])
+
+
+# ------------------------------------------------------------ ZeRO-sharded step
+
+def _zero_kernels():
+    """CPU stand-ins of the library calls, written with the float64 oracle."""
+    from oracle import muon_oracle
+
+    class K:
+        def momentum(self, items, mu, nesterov):
+            for M, G, N in items:
+                Mn = muon_oracle.momentum(M.double().numpy(), G.double().numpy(), mu)
+                Nn = muon_oracle.nesterov(Mn, G.double().numpy(), mu) if nesterov else Mn
+                M.copy_(torch.from_numpy(Mn))
+                N.copy_(torch.from_numpy(Nn))
+
+        def orthogonalize(self, pairs, precision, schedule, eps):
+            for X, O in pairs:
+                O.copy_(torch.from_numpy(muon_oracle.ns_orthogonalize(X.double().numpy())))
+
+        def update(self, items, lr, wd, gamma):
+            for W, O, (n, m) in items:
+                On = muon_oracle.rescale(O.double().numpy(), n, m, gamma)
+                W.copy_(torch.from_numpy(muon_oracle.decay_and_update(W.double().numpy(), On, lr, wd)))
+
+    return K()
+
+
+def _zero_step(rank, world, out_dir):
+    from muon_step_b200.distributed import ZeroMuon
+
+    opt = ZeroMuon(SHAPES, device="cpu", kernels=_zero_kernels())
+    opt.load_weights([W for W, _, _ in _inputs()])
+    for step in range(2):
+        grads = _inputs(seed=100 + 10 * step + rank)  # each rank its own local gradient
+        for k in range(len(SHAPES)):
+            opt.grad(k).copy_(grads[k][1])
+        opt.step(**HYPER)
+    torch.save({"W": [opt.weight(k).clone() for k in range(len(SHAPES))],
+                "M": [s.clone() for s in opt.momentum_shards]},
+               os.path.join(out_dir, f"z{rank}.pt"))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_zero_sharded_step_matches_the_oracle(tmp_path, world):
+    """Reduce-scatter, shard momentum, gather, Newton-Schulz, shard update and
+    all-gather over gloo ranks equal the oracle's step on the summed gradient;
+    every rank ends with the same weights; the momentum shards tile the
+    oracle's momentum."""
+    from muon_step_b200.distributed import shard_size
+    from oracle import muon_oracle
+
+    _run(world, _zero_step, str(tmp_path))
+    outs = [torch.load(tmp_path / f"z{r}.pt") for r in range(world)]
+    W = [w.double().numpy() for w, _, _ in _inputs()]
+    M = [np.zeros(s) for s in SHAPES]
+    for step in range(2):
+        G = [sum(_inputs(seed=100 + 10 * step + r)[k][1].double().numpy() for r in range(world))
+             for k in range(len(SHAPES))]
+        for k in range(len(SHAPES)):
+            W[k], M[k], _ = muon_oracle.muon_step(W[k], G[k], M[k], lr=HYPER["lr"],
+                                                  mu=HYPER["momentum"], wd=HYPER["weight_decay"],
+                                                  gamma=HYPER["gamma"])
+    for k, (n, m) in enumerate(SHAPES):
+        for out in outs:
+            assert torch.equal(out["W"][k], outs[0]["W"][k])
+        # float32 buffers between the float64 pieces
+        assert np.abs(outs[0]["W"][k].double().numpy() - W[k]).max() <= 1e-6 * np.abs(W[k]).max()
+        s = shard_size(n * m, world)
+        flat = torch.cat([outs[r]["M"][k] for r in range(world)])
+        assert flat.numel() == s * world
+        assert np.abs(flat[: n * m].double().numpy() - M[k].reshape(-1)).max() <= 1e-6 * np.abs(M[k]).max()
+        assert not flat[n * m:].any()  # padding stays zero
+
+
+def test_shard_sizes():
+    from muon_step_b200.distributed import shard_size
+    for numel in (1, 3, 4, 5, 1000, 4096, 12345):
+        for world in (1, 2, 3, 8):
+            s = shard_size(numel, world)
+            assert s % 4 == 0 and s * world >= numel and (s - 4) * world < numel

@@ -251,3 +251,44 @@ def test_diagnostics(precision, scale_mode):
             own = h["gamma"] * r
         assert abs(got[k, 1] - own) <= 1e-5 * own, (k, got[k, 1], own)
         assert abs(got[k, 1] - rms_o) <= tol_o(precision, (n, m)) * rms_o, (k, got[k, 1], rms_o)
+
+
+def test_zero_sharded_step_world_one_matches_plan():
+    """ZeroMuon on an NCCL group of one rank (shard kernels, ns_orthogonalize,
+    in-place gathers) equals the single-GPU plan bit for bit: both run the
+    same fp32 operations on the same values."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    import muon_step_b200 as ms
+    from muon_step_b200.distributed import ZeroMuon
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        shapes = [(300, 500), (500, 300), (64, 64), (33, 7)]
+        a = workloads.make_random(shapes, device="cuda", seed=37)
+        b = workloads.make_random(shapes, device="cuda", seed=37)
+        opt = ZeroMuon(shapes)
+        opt.load_weights([a.W[k] for k in range(a.count)])
+        for k in range(a.count):
+            opt.momentum_shards[k][: a.M[k].numel()].copy_(a.M[k].reshape(-1))
+        plan = ms.MuonPlan([(b.W[k], b.G[k], b.M[k]) for k in range(b.count)])
+        for _ in range(2):
+            for k in range(a.count):
+                opt.grad(k).copy_(a.G[k])
+            opt.step()
+            plan.execute()
+        torch.cuda.synchronize()
+        assert ms.sync_status() == 0
+        for k, (n, m) in enumerate(shapes):
+            assert torch.equal(opt.weight(k), b.W[k]), k
+            assert torch.equal(opt.momentum_shards[k][: n * m].view(n, m), b.M[k]), k
+    finally:
+        dist.destroy_process_group()
