@@ -150,6 +150,16 @@ MUON_API muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mod
  * matrices larger than 128 x 128. Muon-step plans only. */
 MUON_API muon_status_t muon_plan_set_diagnostics(muon_plan_t plan, float* out);
 
+/* L2 batching of the Newton-Schulz stages (off by default; 0 turns it off).
+ * With `bytes` > 0, later executes run all steps of the schedule batch by
+ * batch, a batch being consecutive matrices of the plan whose Newton-Schulz
+ * buffers (bf16: 6 r ldc + 4 r ldr bytes per matrix) add up to at most
+ * `bytes` (at least one matrix). With a budget below the L2 size (126 MB on
+ * B200) a batch's buffers stay in L2 across its 3 x steps launches; the
+ * price is 3 x steps launches per batch. The workspace and the results do
+ * not change. Timing events must be set again afterwards. */
+MUON_API muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes);
+
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */
 MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes);
 

@@ -189,6 +189,13 @@ class MuonPlan(_PlanBase):
         _check(_lib.load().muon_plan_set_scale_mode(self._plan, self.SCALE_MODES[mode]),
                "muon_plan_set_scale_mode")
 
+    def set_l2_batching(self, nbytes: int):
+        """Run the Newton-Schulz stages batch by batch, each batch's buffers
+        at most `nbytes` (0: one pass over every matrix). Results and the
+        workspace are unchanged; timing events must be set again."""
+        _check(_lib.load().muon_plan_set_l2_batching(self._plan, int(nbytes)),
+               "muon_plan_set_l2_batching")
+
     def set_diagnostics(self, out: Optional[torch.Tensor]):
         """Write per-matrix diagnostics on every later execute into `out`, a
         float32 CUDA tensor of shape (count, 2): column 0 = ||N||_F (the

@@ -125,6 +125,10 @@ struct muon_plan_s {
   int sumsq_per_tile = 1;           // sum-of-squares slots per Apply tile (unit-RMS scale)
   size_t off_sumsq = 0, off_factor = 0;
   float* diag = nullptr;            // caller's diagnostics output (2 floats per matrix) or NULL
+  // L2 batching: the stage launches run batch by batch over consecutive
+  // matrices whose Newton-Schulz working set fits the budget (0: one batch)
+  size_t l2_batch_bytes = 0;
+  std::vector<std::pair<int, int>> batches;  // internal matrix ranges [first, last)
   std::vector<uint8_t> blob;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
@@ -151,16 +155,59 @@ muon_status_t set_schedule(muon_plan_s* p, const muon_ns_schedule_t* s) {
   return MUON_OK;
 }
 
-// The launch list of one execute (depends on the scale mode).
+// Workspace bytes one matrix's Newton-Schulz buffers take (the L2 working
+// set of its stages): bf16 iterate high x 2 + low, A and B.
+double ns_bytes(const muon_plan_s* p, const MatDesc& md) {
+  const GroupDesc& gd = p->groups[md.group];
+  if (gd.small) return 0.0;
+  const double x = static_cast<double>(gd.r) * gd.ldc, a = static_cast<double>(gd.r) * gd.ldr;
+  return p->prec == MUON_NS_BF16 ? 6.0 * x + 4.0 * a : 8.0 * x + 8.0 * a;
+}
+
+// Split the matrices (internal order) into batches for the stage launches.
+void make_batches(muon_plan_s* p) {
+  p->batches.clear();
+  const int nm = static_cast<int>(p->mats.size());
+  if (p->l2_batch_bytes == 0) {
+    p->batches.emplace_back(0, nm);
+    return;
+  }
+  int first = 0;
+  double acc = 0.0;
+  for (int i = 0; i < nm; ++i) {
+    const double b = ns_bytes(p, p->mats[i]);
+    if (i > first && acc + b > static_cast<double>(p->l2_batch_bytes)) {
+      p->batches.emplace_back(first, i);
+      first = i;
+      acc = 0.0;
+    }
+    acc += b;
+  }
+  p->batches.emplace_back(first, nm);
+}
+
+// First tile of internal matrix i in stage kind k's table (the total for i = count).
+int64_t first_tile(const muon_plan_s* p, int i, int k) {
+  if (i >= static_cast<int>(p->mats.size())) return p->stage_tiles[k];
+  const MatDesc& md = p->mats[i];
+  const GroupDesc& gd = p->groups[md.group];
+  return gd.tile_base[k] + static_cast<int64_t>(md.index) * gd.tiles_per_mat[k];
+}
+
+// The launch list of one execute (depends on the scale mode and the batches).
 void make_launch_list(muon_plan_s* p) {
   const bool unit = p->scale_mode == MUON_SCALE_UNIT_RMS;
+  make_batches(p);
   p->launch_kinds.assign(1, 0);
   if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
   if (p->stage_tiles[kApply] > 0) {
-    for (int k = 0; k < p->steps; ++k) {
-      p->launch_kinds.push_back(1);
-      p->launch_kinds.push_back(2);
-      p->launch_kinds.push_back(k + 1 == p->steps && !unit ? 4 : 3);
+    for (const auto& bt : p->batches) {
+      if (first_tile(p, bt.first, kApply) == first_tile(p, bt.second, kApply)) continue;
+      for (int k = 0; k < p->steps; ++k) {
+        p->launch_kinds.push_back(1);
+        p->launch_kinds.push_back(2);
+        p->launch_kinds.push_back(k + 1 == p->steps && !unit ? 4 : 3);
+      }
     }
     if (unit) {
       p->launch_kinds.push_back(6);
@@ -583,7 +630,11 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   if (plan->stage_tiles[kApply] == 0) return MUON_OK;
   const bool unit = plan->scale_mode == MUON_SCALE_UNIT_RMS;
   const bool diag = plan->mode == 0 && plan->diag != nullptr;
+  // one pass of every step per batch: a batch's buffers stay in L2 across its
+  // 3 x steps launches when the batch fits
+  for (const auto& bt : plan->batches)
   for (int k = 0; k < plan->steps; ++k) {
+    if (first_tile(plan, bt.first, kApply) == first_tile(plan, bt.second, kApply)) break;
     for (int kind = 0; kind < kNumKinds; ++kind) {
       StageArgs sa{};
       sa.groups = groups;
@@ -593,7 +644,8 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       sa.ws = ws;
       sa.scale = scale;
       sa.err = err;
-      sa.total_tiles = plan->stage_tiles[kind];
+      sa.tile_begin = first_tile(plan, bt.first, kind);
+      sa.total_tiles = first_tile(plan, bt.second, kind);
       sa.ngroups = static_cast<int32_t>(plan->groups.size());
       const bool last = k == plan->steps - 1;
       sa.first = k == 0;
@@ -616,7 +668,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
         sa.gamma = hyper->gamma;
       }
       sa.wait_limit_ns = limit;
-      const int64_t tiles = sa.total_tiles;
+      const int64_t tiles = sa.total_tiles - sa.tile_begin;
       cudaError_t e;
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
       if (tc) {
@@ -668,6 +720,14 @@ muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode)
   if (mode != MUON_SCALE_SHAPE && mode != MUON_SCALE_UNIT_RMS && mode != MUON_SCALE_NONE)
     return MUON_ERR_INVALID_ARG;
   plan->scale_mode = mode;
+  make_launch_list(plan);
+  plan->events.clear();  // the launch list may have changed: timing must be set again
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  plan->l2_batch_bytes = bytes;
   make_launch_list(plan);
   plan->events.clear();  // the launch list may have changed: timing must be set again
   return MUON_OK;

@@ -14,8 +14,8 @@
 // significant bits; in fp32 mode as fp32.
 //
 // HBM-bound: each element reads G and M (8 B) and writes M and the two bf16
-// parts (8 B; fp32 mode: M and the fp32 iterate). Tiles are 32 x 128 elements; a tile's threads
-// read and write whole 128-byte lines. When the iterate is the transpose, the
+// parts (8 B; fp32 mode: M and the fp32 iterate). Tiles are 64 x 128 elements; a tile's threads
+// read and write whole 128-byte lines (64 x 128 elements). When the iterate is the transpose, the
 // tile is staged in shared memory so that the transposed writes stay
 // coalesced. Per-tile partial sums of squares go to a buffer; the last tile of
 // each matrix to finish (arrival counter) adds them in a fixed order, in
@@ -183,16 +183,30 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
   }
 
   if (transposed) {
-    // iterate row j = caller column, iterate column i = caller row
+    // iterate row j = caller column, iterate columns i, i + 1 = caller rows:
+    // each lane writes two consecutive elements, a warp 64 of one iterate row
+    static_assert(kEwRows == 64, "two caller rows per lane");
     __syncthreads();
     const int w = tid >> 5, lane = tid & 31;
-    const int64_t i = row0 + lane;
+    const int64_t i = row0 + 2 * lane;
 #pragma unroll 4
     for (int q = 0; q < kEwCols / 8; ++q) {
       const int cc = w * (kEwCols / 8) + q;
       const int64_t j = col0 + cc;
-      if (j < m && i < n) {
-        put(j * ldc + i, stage[lane][cc]);
+      if (j >= m || i >= n) continue;
+      const float v0 = stage[2 * lane][cc], v1 = stage[2 * lane + 1][cc];
+      const int64_t xo = j * ldc + i;  // even: 4-byte aligned pairs (8 bytes in fp32)
+      if (i + 1 < n) {
+        if (a.split) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+          const float2 fh = __bfloat1622float2(h);
+          *reinterpret_cast<__nv_bfloat162*>(xb + xo) = h;
+          *reinterpret_cast<__nv_bfloat162*>(xl + xo) = __floats2bfloat162_rn(v0 - fh.x, v1 - fh.y);
+        } else {
+          *reinterpret_cast<float2*>(xf + xo) = make_float2(v0, v1);
+        }
+      } else {
+        put(xo, v0);
       }
     }
   }

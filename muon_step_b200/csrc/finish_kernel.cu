@@ -11,7 +11,7 @@
 //                       order (double) and stores gamma / RMS(O') (0 when
 //                       O' = 0);
 //   finish_kernel       W <- W (1 - lr wd) - lr factor O' (and O = O'), over
-//                       32 x 128 tiles of the caller's matrix; when the
+//                       64 x 128 tiles of the caller's matrix; when the
 //                       iterate is the transpose, the tile is read through
 //                       shared memory so every global access stays coalesced.
 //
@@ -85,37 +85,45 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
   const UpdateConsts uc = update_consts_raw(a.lr, a.wd, a.factor[mat], gd.c, kScaleNone);
 
   if (md.transposed) {
-    // O'(caller i, j) is iterate element (j, i): read iterate rows j, 32
-    // consecutive i per warp access
+    // O'(caller i, j) is iterate element (j, i): read iterate rows j, two
+    // consecutive i per lane, 64 per warp access
+    static_assert(kEwRows == 64, "two caller rows per lane");
     const int w = tid >> 5, lane = tid & 31;
-    const int64_t i = row0 + lane;
+    const int64_t i = row0 + 2 * lane;
 #pragma unroll 4
     for (int q = 0; q < kEwCols / 8; ++q) {
       const int cc = w * (kEwCols / 8) + q;
       const int64_t j = col0 + cc;
-      stage[lane][cc] = (i < n && j < m) ? o_at(j * ldc + i) : 0.f;
+      const bool jin = j < m;
+      stage[2 * lane][cc] = (i < n && jin) ? o_at(j * ldc + i) : 0.f;
+      stage[2 * lane + 1][cc] = (i + 1 < n && jin) ? o_at(j * ldc + i + 1) : 0.f;
     }
     __syncthreads();
   }
-  // caller element (row, col): thread -> one column, rows (tid / 128) + 2 k
-  constexpr int R = kEwRows / 2;
+  // caller element (row, col): thread -> one column, rows (tid / 128) + 2 k,
+  // in two halves of the tile (loads of a half before its stores)
+  constexpr int R = kEwRows / 4;
   const int cc = tid & (kEwCols - 1);
   const int64_t col = col0 + cc;
-  float o[R], w[R];
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    const int r0 = half * (kEwRows / 2) + (tid >> 7);
+    float o[R], w[R];
 #pragma unroll
-  for (int k = 0; k < R; ++k) {
-    const int rr = (tid >> 7) + 2 * k;
-    const int64_t row = row0 + rr;
-    const bool in = row < n && col < m;
-    o[k] = !in ? 0.f : (md.transposed ? stage[rr][cc] : o_at(row * ldc + col));
-    w[k] = (in && md.W) ? md.W[row * m + col] : 0.f;
-  }
+    for (int k = 0; k < R; ++k) {
+      const int rr = r0 + 2 * k;
+      const int64_t row = row0 + rr;
+      const bool in = row < n && col < m;
+      o[k] = !in ? 0.f : (md.transposed ? stage[rr][cc] : o_at(row * ldc + col));
+      w[k] = (in && md.W) ? md.W[row * m + col] : 0.f;
+    }
 #pragma unroll
-  for (int k = 0; k < R; ++k) {
-    const int64_t row = row0 + (tid >> 7) + 2 * k;
-    if (row >= n || col >= m) continue;
-    if (md.O) md.O[row * m + col] = o[k];
-    if (md.W) md.W[row * m + col] = fmaf(w[k], uc.keep, -uc.step * o[k]);
+    for (int k = 0; k < R; ++k) {
+      const int64_t row = row0 + r0 + 2 * k;
+      if (row >= n || col >= m) continue;
+      if (md.O) md.O[row * m + col] = o[k];
+      if (md.W) md.W[row * m + col] = fmaf(w[k], uc.keep, -uc.step * o[k]);
+    }
   }
 }
 

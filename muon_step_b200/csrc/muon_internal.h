@@ -30,8 +30,10 @@ constexpr int kSBM = 64;
 constexpr int kSBN = 64;
 constexpr int kSBK = 16;
 
-// elementwise (momentum / norm / cast) tile: 32 rows x 128 columns.
-constexpr int kEwRows = 32;
+// elementwise (momentum / norm / cast) tile: 64 rows x 128 columns. 64 rows
+// make the transposed writes of the bf16 iterate parts whole 128-byte lines
+// (two caller rows per lane).
+constexpr int kEwRows = 64;
 constexpr int kEwCols = 128;
 
 enum StageKind : int { kGram = 0, kPoly = 1, kApply = 2, kNumKinds = 3 };
@@ -99,6 +101,7 @@ struct StageArgs {
   char* ws;               // workspace base
   const float* scale;     // per-matrix 1 / (||N||_F + eps)
   int* err;               // device error word
+  int64_t tile_begin;     // this launch walks tiles [tile_begin, total_tiles) of the kind's table
   int64_t total_tiles;
   int32_t ngroups;
   int32_t first;          // first Newton-Schulz step: fold the normalisation scale

@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) stage_simt_kernel(const __grid_constant__
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;
 
-  for (int64_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
+  for (int64_t t = a.tile_begin + blockIdx.x; t < a.total_tiles; t += gridDim.x) {
     const int g = stage_group<KIND>(a, t);
     const GroupDesc& gd = a.groups[g];
     const int64_t local = t - gd.tile_base[KIND];
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(256) stage_simt_kernel(const __grid_constant__
 
 cudaError_t launch_stage_simt(StageKind kind, const StageArgs& args, int grid,
                               cudaStream_t stream) {
-  if (args.total_tiles <= 0) return cudaSuccess;
+  if (args.total_tiles <= args.tile_begin) return cudaSuccess;
   switch (kind) {
     case kGram: stage_simt_kernel<kGram><<<grid, 256, 0, stream>>>(args); break;
     case kPoly: stage_simt_kernel<kPoly><<<grid, 256, 0, stream>>>(args); break;

@@ -500,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
     for (int i = 0; i < kStages; ++i) leader_full[i] = ptx::mapa_shared(ptx::smem_u32(&s.full[i]), 0);
     uint32_t stage = 0, phase = 0;
     bool ok = true;
-    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
+    for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
       const int bz = static_cast<int>(tc.b);
       for (int kb = 0; kb < tc.kblocks; ++kb) {
@@ -548,7 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
     bool ok = true;
     bool issued = false;
-    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
+    for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
       if (!ptx::mbar_wait(&s.tempty[acc], acc_phase ^ 1, limit, s.abort_flag)) {
         raise_abort(a, s);
@@ -613,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
     constexpr int kReuseWait = S - 1 - D;  // store groups that may still be pending
     uint32_t acc = 0, acc_phase = 0;
     bool ok = true;
-    for (int64_t t = pair; ok && t < a.total_tiles; t += npairs) {
+    for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
       const GroupDesc& gd = a.groups[tc.g];
       const int row0 = tc.I * kPairTile + static_cast<int>(rank) * kHalf + quarter * 32;
@@ -754,7 +754,7 @@ cudaError_t launch_kind(const StageArgs& args, int grid, cudaStream_t stream) {
 size_t stage_tc_smem_bytes() { return Cfg<kGram>::kSmem; }
 
 cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, cudaStream_t stream) {
-  if (args.total_tiles <= 0) return cudaSuccess;
+  if (args.total_tiles <= args.tile_begin) return cudaSuccess;
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidConfiguration;
   switch (kind) {
     case kGram: return launch_kind<kGram>(args, grid, stream);

@@ -126,7 +126,7 @@ def expected_workspace(shapes, prec):
         groups.setdefault(key, []).append((n, m))
     al = lambda x, a: (x + a - 1) // a * a
     ng, nm = len(groups), len(shapes)
-    ew = sum(math.ceil(n / 32) * math.ceil(m / 128) for n, m in shapes)
+    ew = sum(math.ceil(n / 64) * math.ceil(m / 128) for n, m in shapes)
     off = al(ng * 160, 256)          # GroupDesc is 160 bytes
     off = al(off + nm * 88, 256)     # MatDesc is 88 bytes
     off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
@@ -301,3 +301,33 @@ def test_shard_calls_validate_before_touching_a_device(lib):
     upd[0] = ShardUpdate(FAKE, FAKE + 4096, 16, 4, 4)
     assert lib.muon_shard_update(upd, 1, float("inf"), 0.1, 0.2, ws, 1 << 20, None) == MUON_ERR_INVALID_ARG
     assert lib.muon_shard_update(upd, 1, 0.02, 0.1, 0.2, ws, 16, None) == MUON_ERR_WORKSPACE
+
+
+def test_l2_batching_repeats_the_stage_launches_per_batch(lib):
+    shapes = [(300, 400), (400, 300), (300, 400), (64, 64)]
+    st, plan = create(lib, shapes)
+    assert st == MUON_OK
+    cnt = ctypes.c_int()
+    kinds = (ctypes.c_int * 512)()
+
+    def kinds_now():
+        assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 512) == MUON_OK
+        return list(kinds[:cnt.value])
+
+    one_pass = [1, 2, 3] * 9 + [1, 2, 4]
+    assert kinds_now() == [0, 5] + one_pass
+    ws0 = ctypes.c_size_t()
+    assert lib.muon_plan_workspace_size(plan, ctypes.byref(ws0)) == MUON_OK
+    # one 300 x 400 matrix needs 6*300*400 + 4*300*304 = 1,084,800 bytes of buffers
+    assert lib.muon_plan_set_l2_batching(plan, 1_200_000) == MUON_OK
+    assert kinds_now() == [0, 5] + one_pass * 3
+    assert lib.muon_plan_set_l2_batching(plan, 2 * 1_084_800) == MUON_OK
+    assert kinds_now() == [0, 5] + one_pass * 2
+    assert lib.muon_plan_set_l2_batching(plan, 1) == MUON_OK  # at least one matrix per batch
+    assert kinds_now() == [0, 5] + one_pass * 3
+    ws1 = ctypes.c_size_t()
+    assert lib.muon_plan_workspace_size(plan, ctypes.byref(ws1)) == MUON_OK
+    assert ws1.value == ws0.value
+    assert lib.muon_plan_set_l2_batching(plan, 0) == MUON_OK
+    assert kinds_now() == [0, 5] + one_pass
+    lib.muon_plan_destroy(plan)

@@ -292,3 +292,25 @@ def test_zero_sharded_step_world_one_matches_plan():
             assert torch.equal(opt.momentum_shards[k][: n * m].view(n, m), b.M[k]), k
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_l2_batching_gives_identical_results(precision):
+    """Batch-by-batch stage launches compute every tile as one pass does."""
+    import muon_step_b200 as ms
+
+    shapes = [(300, 520), (520, 300), (64, 64), (257, 129), (300, 520), (100, 37)]
+    a = workloads.make_random(shapes, device="cuda", seed=41)
+    b = workloads.make_random(shapes, device="cuda", seed=41)
+    Oa = [torch.empty_like(w) for w in a.W]
+    Ob = [torch.empty_like(w) for w in b.W]
+    pa = ms.MuonPlan([(a.W[k], a.G[k], a.M[k], Oa[k]) for k in range(a.count)], precision=precision)
+    pb = ms.MuonPlan([(b.W[k], b.G[k], b.M[k], Ob[k]) for k in range(b.count)], precision=precision)
+    pb.set_l2_batching(1)  # one matrix per batch
+    for _ in range(2):
+        pa.execute()
+        pb.execute()
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for k in range(a.count):
+        assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k]) and torch.equal(Oa[k], Ob[k])
