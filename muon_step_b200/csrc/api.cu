@@ -194,6 +194,24 @@ int64_t first_tile(const muon_plan_s* p, int i, int k) {
   return gd.tile_base[k] + static_cast<int64_t>(md.index) * gd.tiles_per_mat[k];
 }
 
+// Gram, Poly and the last Apply take the eight-epilogue-warp variant when the
+// tile-weighted mean length of their main loops (K = c for Gram, r for the
+// others) is at most 512 (1024 for the last Apply, whose epilogue also moves
+// W): there the epilogue, not the operand feed, sets the tile rate. Measured
+// on 512^2, 512 x 2048, 1024^2 and 2048^2 batches.
+bool wide_epilogue(const muon_plan_s* p, const std::pair<int, int>& bt, int kind, bool last) {
+  if (kind == kApply && !last) return true;
+  const double kmax = (kind == kApply) ? 1024.0 : 512.0;
+  double tiles = 0.0, ksum = 0.0;
+  for (int i = bt.first; i < bt.second; ++i) {
+    const GroupDesc& gd = p->groups[p->mats[i].group];
+    const double t = static_cast<double>(gd.tiles_per_mat[kind]);
+    tiles += t;
+    ksum += t * (kind == kGram ? gd.c : gd.r);
+  }
+  return tiles > 0.0 && ksum <= kmax * tiles;
+}
+
 // The launch list of one execute (depends on the scale mode and the batches).
 void make_launch_list(muon_plan_s* p) {
   const bool unit = p->scale_mode == MUON_SCALE_UNIT_RMS;
@@ -329,7 +347,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   p->off_scale = off;
   off = align_up(off + nm * sizeof(float), 256);
   // unit-RMS scale: sums of squares of O' per Apply tile, then gamma / RMS per matrix
-  p->sumsq_per_tile = tc ? 8 : 1;  // tensor cores: 2 CTAs x 4 epilogue warps per tile
+  p->sumsq_per_tile = tc ? 16 : 1;  // tensor cores: 2 CTAs x 8 slots (one per epilogue warp) per tile
   p->off_sumsq = off;
   off = align_up(off + static_cast<size_t>(p->stage_tiles[kApply]) * p->sumsq_per_tile * sizeof(float), 256);
   p->off_factor = off;
@@ -673,7 +691,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
       if (tc) {
         const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, sms / 2));
-        e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, stream);
+        e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, wide_epilogue(plan, bt, kind, sa.last != 0), stream);
       } else {
         const int grid = static_cast<int>(std::min<int64_t>(tiles, 8LL * sms));
         e = launch_stage_simt(static_cast<StageKind>(kind), sa, grid, stream);

@@ -14,7 +14,9 @@ cudaError_t launch_elementwise(const EwArgs& args, cudaStream_t stream);
 
 // One Newton-Schulz stage over every matrix of the plan, bf16 operands on
 // the tcgen05 tensor cores (TMA -> shared memory -> MMA -> TMEM -> epilogue).
-cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid,
+// `wide`: Gram, Poly or ApplyLast with eight epilogue warps (short main loops);
+// Apply always has eight
+cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, bool wide,
                             cudaStream_t stream);
 
 // Every Newton-Schulz step and the update for the small matrices, one CTA

@@ -77,25 +77,34 @@ constexpr size_t kBarrierBytes = 512;
 constexpr int kTmapBytes = 128;
 
 // Per-kind layout: ring depth and the epilogue staging slots (kEpiSlots per
-// warp, four epilogue warps, one per TMEM lane quarter). The Apply-like kinds
-// load an input per 32 x 32 chunk and keep kEpiSlots - 1 of those loads in
-// flight ahead of the chunk being processed; their epilogue, not the main
-// loop, sets the tile rate when the loads come from HBM. Slot sizes:
+// warp; four epilogue warps, one per TMEM lane quarter, or eight for Apply,
+// two per quarter). The Apply-like kinds load an input per 32 x 32 chunk
+// ahead of the chunk being processed. Slot sizes:
 //   Gram       [bf16 out | bf16 mirror out]                            4 KB
 //   Poly       [bf16 A in | bf16 out | bf16 mirror out]                6 KB
 //   Apply      [bf16 iterate high in / out | bf16 low in / out]        4 KB
 //   ApplyLast  [bf16 high in | bf16 low in, then fp32 O out | fp32 W in / out]  8 KB
 // The iterate is kept as two bf16 parts, X = high + low (16 significant
 // bits); the high part is the tensor-core operand.
-template <int KIND>
+//
+// Wide variants run eight epilogue warps, two per TMEM lane quarter, each
+// taking half of the columns, for one ring stage less. Apply is always wide
+// (its epilogue moves the most data); Gram, Poly and ApplyLast are wide when
+// the plan's tiles have short main loops, where the epilogue sets the tile
+// rate (the host picks, by the mean K of the launch's tiles).
+template <int KIND, bool WIDE = false>
 struct Cfg {
-  static constexpr int kEpiWarps = 4;
+  static constexpr bool kWide = WIDE || KIND == kApply;
+  static constexpr int kEpiWarps = kWide ? 8 : 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  static constexpr int kStages = (KIND == kGram) ? 6 : (KIND == kApplyLast) ? 4 : 5;
+  static constexpr int kStages = (KIND == kGram)   ? (kWide ? 5 : 6)
+                                 : (KIND == kPoly) ? (kWide ? 4 : 5)
+                                 : (KIND == kApply) ? 5
+                                                    : (kWide ? 3 : 4);
   static constexpr int kSlot = (KIND == kApplyLast) ? 2 * kEpiF32
                                : (KIND == kPoly)    ? 3 * kEpiB16
                                                     : 2 * kEpiB16;
-  static constexpr int kEpiSlots = (KIND == kApply) ? 4 : (KIND == kApplyLast) ? 3 : 2;
+  static constexpr int kEpiSlots = (KIND == kApplyLast && !kWide) ? 3 : 2;
   static constexpr int kEpiBytes = kEpiWarps * kEpiSlots * kSlot;
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kEpiBytes + kBarrierBytes;
   static constexpr bool kApplyLike = (KIND == kApply || KIND == kApplyLast);
@@ -107,6 +116,7 @@ struct Cfg {
 };
 
 constexpr int kOffLow = kEpiB16;   // low part of the iterate in Apply-like slots
+constexpr int kSumsqSlots = 8;     // sum-of-squares slots per CTA and tile (most epilogue warps)
 constexpr int kOffLastW = kEpiF32;
 
 constexpr uint32_t kIdescKK = ptx::idesc_bf16(kPairTile, kPairTile, 0, 0);   // both K-major
@@ -188,20 +198,20 @@ struct Smem {
   volatile int* abort_flag;
 };
 
-template <int KIND>
+template <typename C>
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.ring = base;
-  s.epi = base + Cfg<KIND>::kStages * kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.epi + Cfg<KIND>::kEpiBytes);
+  s.epi = base + C::kStages * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.epi + C::kEpiBytes);
   s.full = bars;
-  s.empty = s.full + Cfg<KIND>::kStages;
-  s.tfull = s.empty + Cfg<KIND>::kStages;
+  s.empty = s.full + C::kStages;
+  s.tfull = s.empty + C::kStages;
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
   s.eload = s.drain + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + Cfg<KIND>::kEpiSlots * Cfg<KIND>::kEpiWarps);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + C::kEpiSlots * C::kEpiWarps);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
   return s;
 }
@@ -451,14 +461,14 @@ __device__ __forceinline__ void epi_apply_last(const StageArgs& a, const GroupDe
 
 // -------------------------------------------------------------- kernel
 
-template <int KIND>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads, 1)
+template <int KIND, bool WIDE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND, WIDE>::kThreads, 1)
     stage_tc_kernel(const __grid_constant__ StageArgs a) {
-  using C = Cfg<KIND>;
+  using C = Cfg<KIND, WIDE>;
   constexpr int kStages = C::kStages;
   constexpr int kEpiWarps = C::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
-  const Smem s = carve<KIND>(smem_raw);
+  const Smem s = carve<C>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
@@ -709,7 +719,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
         // one slot per (tile, CTA of the pair, epilogue warp); every slot is written
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
-        if (lane == 0) a.sumsq[(t * 2 + rank) * kEpiWarps + ew] = ssq;
+        // kSumsqSlots per CTA and tile; a kind with fewer epilogue warps zeroes the rest
+        if (lane == 0) {
+          float* dst = a.sumsq + (t * 2 + rank) * kSumsqSlots;
+          dst[ew] = ssq;
+          for (int e = ew + kEpiWarps; e < kSumsqSlots; e += kEpiWarps) dst[e] = 0.f;
+        }
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -738,14 +753,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<KIND>::kThreads,
   }
 }
 
-template <int KIND>
+template <int KIND, bool WIDE>
 cudaError_t launch_kind(const StageArgs& args, int grid, cudaStream_t stream) {
-  constexpr size_t smem = Cfg<KIND>::kSmem;
+  using C = Cfg<KIND, WIDE>;
+  constexpr size_t smem = C::kSmem;
   static_assert(smem <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(stage_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(stage_tc_kernel<KIND, WIDE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  stage_tc_kernel<KIND><<<grid, Cfg<KIND>::kThreads, smem, stream>>>(args);
+  stage_tc_kernel<KIND, WIDE><<<grid, C::kThreads, smem, stream>>>(args);
   return cudaGetLastError();
 }
 
@@ -753,14 +769,19 @@ cudaError_t launch_kind(const StageArgs& args, int grid, cudaStream_t stream) {
 
 size_t stage_tc_smem_bytes() { return Cfg<kGram>::kSmem; }
 
-cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, cudaStream_t stream) {
+cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, bool wide,
+                            cudaStream_t stream) {
   if (args.total_tiles <= args.tile_begin) return cudaSuccess;
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidConfiguration;
   switch (kind) {
-    case kGram: return launch_kind<kGram>(args, grid, stream);
-    case kPoly: return launch_kind<kPoly>(args, grid, stream);
+    case kGram:
+      return wide ? launch_kind<kGram, true>(args, grid, stream) : launch_kind<kGram, false>(args, grid, stream);
+    case kPoly:
+      return wide ? launch_kind<kPoly, true>(args, grid, stream) : launch_kind<kPoly, false>(args, grid, stream);
     case kApply:
-      return args.last ? launch_kind<kApplyLast>(args, grid, stream) : launch_kind<kApply>(args, grid, stream);
+      if (!args.last) return launch_kind<kApply, true>(args, grid, stream);
+      return wide ? launch_kind<kApplyLast, true>(args, grid, stream)
+                  : launch_kind<kApplyLast, false>(args, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }

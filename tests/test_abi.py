@@ -137,11 +137,11 @@ def expected_workspace(shapes, prec):
     off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
-    # unit-RMS scale: sums of squares per Apply tile (8 slots on tensor cores), a factor per matrix
+    # unit-RMS scale: sums of squares per Apply tile (16 slots on tensor cores), a factor per matrix
     if prec == MUON_NS_BF16:
         apply_tiles = sum(len(mem) * math.ceil(r / 256) * math.ceil(c / 256)
                           for (r, c), mem in groups.items() if c > 128)
-        slots = 8
+        slots = 16
     else:
         apply_tiles = sum(len(mem) * math.ceil(r / 64) * math.ceil(c / 64) for (r, c), mem in groups.items())
         slots = 1
