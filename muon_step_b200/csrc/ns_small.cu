@@ -4,13 +4,15 @@
 // kernels would spend their time on padding and per-launch latency (30
 // dependent launches of mostly empty 256 x 256 tiles). Here one CTA of 128
 // threads (thread = iterate row = TMEM lane) runs every step of the schedule
-// for one matrix and then writes the update:
+// for one matrix and then writes the update. 256 threads: thread t owns
+// iterate row t % 128 (its TMEM lane) and half t / 128 of its columns, so
+// each product's epilogue is two 32-column chunks per thread:
 //
 //   shared memory  X, A and B as bf16 128 x 128 tiles in the 128-byte-swizzle
 //                  K-major layout (two 64-column chunks of 128 rows). The
 //                  same X buffer is the K-major operand of the Gram product
 //                  and the MN-major operand of the Apply product.
-//   registers      the fp32 iterate, one row per thread (aX term).
+//   registers      the fp32 iterate, half a row per thread (aX term).
 //   TMEM           one 128-column fp32 accumulator reused by the three
 //                  products: A = X X^T, B = b A + c A A^T, X' = a X + B X
 //                  ("Ch 06 · Muon" §3 and §5 Algorithm 1, regrouped), with
@@ -73,9 +75,12 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const fl
 
 }  // namespace
 
-__global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant__ SmallArgs a) {
+constexpr int kThreads = 256;
+constexpr int kHalfCols = kS / 2;  // columns per thread
+
+__global__ void __launch_bounds__(kThreads, 2) ns_small_kernel(const __grid_constant__ SmallArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float red[4];
+  __shared__ float red[kThreads / 32];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Xs = base;
   uint8_t* As = Xs + kTileBytes;
@@ -87,6 +92,9 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int row = tid & (kS - 1);     // iterate row = TMEM lane
+  const int half = tid >> 7;          // which 64 columns
+  const int ch0 = half * (kHalfCols / 32);  // first 32-column chunk
   if (tid == 0) {
     ptx::mbar_init(bar_ld, 1);
     ptx::mbar_init(bar_mma, 1);
@@ -101,7 +109,8 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lanes
+  // this warp's lanes (warps w and w + 4 share lanes 32 (w % 4) ...)
+  const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
   const uint32_t sX = ptx::smem_u32(Xs), sA = ptx::smem_u32(As), sB = ptx::smem_u32(Bs);
   const uint64_t limit = a.wait_limit_ns;
   uint32_t ld_phase = 0, mma_phase = 0;
@@ -140,17 +149,19 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       ptx::tma_load_3d(Xs, tm, bar_ld, 0, 0, md.index);
       ptx::tma_load_3d(Xs + kChunkBytes, tm, bar_ld, 64, 0, md.index);
     }
-    // iterate row `tid` into fp32 registers, high + low bf16 parts (zero outside the matrix)
-    float x[kS];
-    const int64_t row_off = (static_cast<int64_t>(md.index) * r + tid) * ldc;
+    // this thread's half row of the iterate into fp32 registers, high + low
+    // bf16 parts (zero outside the matrix)
+    float x[kHalfCols];
+    const int col_base = half * kHalfCols;
+    const int64_t row_off = (static_cast<int64_t>(md.index) * r + row) * ldc + col_base;
     const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xb_off[0]) + row_off;
     const __nv_bfloat16* xl = reinterpret_cast<const __nv_bfloat16*>(a.ws + gd.xlo_off) + row_off;
     // 16-byte loads: rows start 16-byte aligned (ldc is a multiple of 8) and
     // the 8-element groups that start below c lie inside the row's ldc
 #pragma unroll
-    for (int q = 0; q < kS / 8; ++q) {
+    for (int q = 0; q < kHalfCols / 8; ++q) {
       uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;
-      if (tid < r && 8 * q < c) {
+      if (row < r && col_base + 8 * q < c) {
         hv = *reinterpret_cast<const uint4*>(xh + 8 * q);
         lv = *reinterpret_cast<const uint4*>(xl + 8 * q);
       }
@@ -161,8 +172,9 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
         const float2 fh = __bfloat1622float2(h2[k]);
         const float2 fl = __bfloat1622float2(l2[k]);
         const int e = 8 * q + 2 * k;
-        x[e] = e < c ? fh.x + fl.x : 0.f;  // columns c .. ldc of the buffers are not written
-        x[e + 1] = e + 1 < c ? fh.y + fl.y : 0.f;
+        // columns c .. ldc of the buffers are not written
+        x[e] = col_base + e < c ? fh.x + fl.x : 0.f;
+        x[e + 1] = col_base + e + 1 < c ? fh.y + fl.y : 0.f;
       }
     }
     if (!ptx::mbar_wait(bar_ld, ld_phase, limit, abort_flag)) {
@@ -187,12 +199,12 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       wait_mma();
       if (!ok) break;
 #pragma unroll
-      for (int ch = 0; ch < kS / 32; ++ch) {
+      for (int ch = ch0; ch < ch0 + kHalfCols / 32; ++ch) {
         float v[32];
         ptx::tmem_ld32(trow + ch * 32, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] *= alpha * alpha;
-        put_row32(As, tid, ch, v);
+        put_row32(As, row, ch, v);
       }
       hand_over();
 
@@ -205,12 +217,12 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       wait_mma();
       if (!ok) break;
 #pragma unroll
-      for (int ch = 0; ch < kS / 32; ++ch) {
+      for (int ch = ch0; ch < ch0 + kHalfCols / 32; ++ch) {
         float v[32];
         ptx::tmem_ld32(trow + ch * 32, v);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const Bf16x8 p = *reinterpret_cast<const Bf16x8*>(As + piece_off(tid, 4 * ch + q));
+          const Bf16x8 p = *reinterpret_cast<const Bf16x8*>(As + piece_off(row, 4 * ch + q));
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const float2 f = __bfloat1622float2(p.v[h]);
@@ -218,7 +230,7 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
             v[8 * q + 2 * h + 1] = fmaf(cb, f.y, cc * v[8 * q + 2 * h + 1]);
           }
         }
-        put_row32(Bs, tid, ch, v);
+        put_row32(Bs, row, ch, v);
       }
       hand_over();
 
@@ -232,15 +244,15 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       if (!ok) break;
       const bool last = (k + 1 == a.steps);
 #pragma unroll
-      for (int ch = 0; ch < kS / 32; ++ch) {
+      for (int j = 0; j < kHalfCols / 32; ++j) {
         float v[32];
-        ptx::tmem_ld32(trow + ch * 32, v);
+        ptx::tmem_ld32(trow + (ch0 + j) * 32, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          x[32 * ch + e] = alpha * fmaf(ca, x[32 * ch + e], v[e]);
-          v[e] = x[32 * ch + e];
+          x[32 * j + e] = alpha * fmaf(ca, x[32 * j + e], v[e]);
+          v[e] = x[32 * j + e];
         }
-        if (!last) put_row32(Xs, tid, ch, v);
+        if (!last) put_row32(Xs, row, ch0 + j, v);
       }
       hand_over();
     }
@@ -253,12 +265,15 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
     // global access one contiguous segment.
     float* T = reinterpret_cast<float*>(As);
 #pragma unroll
-    for (int e = 0; e < kS; ++e) T[tid * kS + (e ^ (tid & 31))] = x[e];
+    for (int e = 0; e < kHalfCols; ++e) {
+      const int col = col_base + e;
+      T[row * kS + (col ^ (row & 31))] = x[e];
+    }
     if (a.scale_mode == kScaleUnitRms || a.diag) {
       // RMS(O') over the matrix (zeros outside it), in a fixed order
       float ssq = 0.f;
 #pragma unroll
-      for (int e = 0; e < kS; ++e) ssq = fmaf(x[e], x[e], ssq);
+      for (int e = 0; e < kHalfCols; ++e) ssq = fmaf(x[e], x[e], ssq);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
       if ((tid & 31) == 0) red[warp] = ssq;
@@ -268,9 +283,10 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       // unit-RMS: O = O' gamma / RMS(O'), a plain scale once RMS is known
       float gam = a.gamma;
       int mode = a.scale_mode;
-      const float rms = (mode == kScaleUnitRms || a.diag)
-                            ? sqrtf((red[0] + red[1] + red[2] + red[3]) / (static_cast<float>(r) * c))
-                            : 0.f;
+      float tot = 0.f;
+      if (mode == kScaleUnitRms || a.diag)
+        for (int w = 0; w < kThreads / 32; ++w) tot += red[w];
+      const float rms = (mode == kScaleUnitRms || a.diag) ? sqrtf(tot / (static_cast<float>(r) * c)) : 0.f;
       if (mode == kScaleUnitRms) {
         gam = rms > 0.f ? a.gamma / rms : 0.f;
         mode = kScaleNone;
@@ -285,25 +301,24 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const __grid_constant_
       const bool tr = md.transposed != 0;
       const int rows = tr ? c : r;  // caller rows
       const int cols = tr ? r : c;  // caller columns
-      for (int row = warp; row < rows; row += 4) {
+      for (int crow = warp; crow < rows; crow += kThreads / 32) {
+        float* Wr = md.W ? md.W + static_cast<int64_t>(crow) * md.m : nullptr;
+        float* Or = md.O ? md.O + static_cast<int64_t>(crow) * md.m : nullptr;
         float w[kS / 32], o[kS / 32];
-        int64_t idx[kS / 32];
-        bool in[kS / 32];
 #pragma unroll
         for (int q = 0; q < kS / 32; ++q) {
           const int col = 32 * q + lane;
-          in[q] = col < cols;
-          const int i = tr ? col : row;  // iterate coordinates of caller (row, col)
-          const int j = tr ? row : col;
+          const int i = tr ? col : crow;  // iterate coordinates of caller (crow, col)
+          const int j = tr ? crow : col;
           o[q] = T[i * kS + (j ^ (i & 31))];
-          idx[q] = static_cast<int64_t>(row) * md.m + col;
-          w[q] = (in[q] && md.W) ? md.W[idx[q]] : 0.f;
+          w[q] = (col < cols && Wr) ? Wr[col] : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < kS / 32; ++q) {
-          if (!in[q]) continue;
-          if (md.O) md.O[idx[q]] = o[q];
-          if (md.W) md.W[idx[q]] = fmaf(w[q], uc.keep, -uc.step * o[q]);
+          const int col = 32 * q + lane;
+          if (col >= cols) continue;
+          if (Or) Or[col] = o[q];
+          if (Wr) Wr[col] = fmaf(w[q], uc.keep, -uc.step * o[q]);
         }
       }
     }
@@ -324,7 +339,7 @@ cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  ns_small_kernel<<<grid, 128, kSmem, stream>>>(args);
+  ns_small_kernel<<<grid, kThreads, kSmem, stream>>>(args);
   return cudaGetLastError();
 }
 
