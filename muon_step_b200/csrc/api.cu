@@ -119,7 +119,9 @@ struct muon_plan_s {
          off_small = 0, off_partial = 0, off_counter = 0, off_scale = 0, desc_bytes = 0,
          ws_bytes = 0;
   std::vector<int32_t> small_mats;  // internal indices run by the small-matrix kernel
-  std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small,
+  std::vector<int32_t> mid_mats;    // internal indices run by the mid-size kernel
+  size_t off_mid = 0;
+  std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small, 8 mid,
                                     // 6 RMS reduction, 7 update pass (unit-RMS scale)
   int scale_mode = MUON_SCALE_SHAPE;
   int sumsq_per_tile = 1;           // sum-of-squares slots per Apply tile (unit-RMS scale)
@@ -218,6 +220,7 @@ void make_launch_list(muon_plan_s* p) {
   make_batches(p);
   p->launch_kinds.assign(1, 0);
   if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
+  if (!p->mid_mats.empty()) p->launch_kinds.push_back(8);
   if (p->stage_tiles[kApply] > 0) {
     for (const auto& bt : p->batches) {
       if (first_tile(p, bt.first, kApply) == first_tile(p, bt.second, kApply)) continue;
@@ -269,7 +272,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     gd.count = static_cast<int32_t>(members[g].size());
     gd.first_mat = static_cast<int32_t>(p->mats.size());
     double fl[kNumKinds] = {0, 0, 0};
-    gd.small = (tc && r <= kSmallMax && c <= kSmallMax) ? 1 : 0;
+    gd.small = (tc && r <= kSmallMax && c <= kSmallMax) ? 1 : (tc && r <= kSmallMax && c <= kMidMaxC) ? 2 : 0;
     if (gd.small) {
       // one CTA per matrix, dense 128 x 128 products; count the useful FLOPs
       fl[kGram] = 2.0 * r * r * static_cast<double>(c);
@@ -316,7 +319,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
       md.flags = 0;
       if (md.W && rows16 && (reinterpret_cast<uintptr_t>(md.W) & 15) == 0) md.flags |= kMatWTma;
       if (md.O && rows16 && (reinterpret_cast<uintptr_t>(md.O) & 15) == 0) md.flags |= kMatOTma;
-      if (gd.small) p->small_mats.push_back(static_cast<int32_t>(p->mats.size()));
+      if (gd.small == 1) p->small_mats.push_back(static_cast<int32_t>(p->mats.size()));
+      if (gd.small == 2) p->mid_mats.push_back(static_cast<int32_t>(p->mats.size()));
       md.ew_tile_begin = ew_total;
       md.ew_tiles = cdiv(md.n, kEwRows) * cdiv(md.m, kEwCols);
       ew_total += md.ew_tiles;
@@ -340,6 +344,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(int32_t), 256);
   p->off_small = off;
   off = align_up(off + p->small_mats.size() * sizeof(int32_t), 256);
+  p->off_mid = off;
+  off = align_up(off + p->mid_mats.size() * sizeof(int32_t), 256);
   p->off_partial = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
   p->off_counter = off;
@@ -389,6 +395,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   std::memcpy(p->blob.data() + p->off_mats, p->mats.data(), nm * sizeof(MatDesc));
   if (!p->small_mats.empty())
     std::memcpy(p->blob.data() + p->off_small, p->small_mats.data(), p->small_mats.size() * sizeof(int32_t));
+  if (!p->mid_mats.empty())
+    std::memcpy(p->blob.data() + p->off_mid, p->mid_mats.data(), p->mid_mats.size() * sizeof(int32_t));
   make_launch_list(p);
   auto* tile_mat = reinterpret_cast<int32_t*>(p->blob.data() + p->off_tile_mat);
   for (size_t k = 0; k < nm; ++k)
@@ -620,7 +628,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   const bool tc = plan->prec == MUON_NS_BF16;
   const int sms = g_num_sms[dev];
   int slot = 2;
-  if (!plan->small_mats.empty()) {
+  if (!plan->small_mats.empty() || !plan->mid_mats.empty()) {
     SmallArgs sm{};
     sm.groups = groups;
     sm.mats = mats;
@@ -640,10 +648,20 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
     sm.diag = plan->mode == 0 ? plan->diag : nullptr;
     sm.wait_limit_ns = limit;
     for (int k = 0; k < 3 * plan->steps; ++k) sm.abc[k] = plan->abc[k];
-    const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
-    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
-    if (launch_small(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
-    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (sm.nsmall > 0) {
+      const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      if (launch_small(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
+    if (!plan->mid_mats.empty()) {
+      sm.small_mats = reinterpret_cast<const int32_t*>(ws + plan->off_mid);
+      sm.nsmall = static_cast<int64_t>(plan->mid_mats.size());
+      const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, static_cast<int64_t>(sms)));
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      if (launch_mid(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
   }
   if (plan->stage_tiles[kApply] == 0) return MUON_OK;
   const bool unit = plan->scale_mode == MUON_SCALE_UNIT_RMS;

@@ -70,11 +70,17 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
   float* xf = reinterpret_cast<float*>(a.ws + gd.xf_off[0]) + md.index * mat_elems;
   __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xb_off[0]) + md.index * mat_elems;
   __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xlo_off) + md.index * mat_elems;
-  auto put = [&](int64_t xo, float v) {
+  const int lo_kind = gd.small;  // layout of the low part (lo_index)
+  // mid-size matrices keep the low part in 8-column groups: it is written
+  // from the staged tile in a second pass, one 16-byte piece per thread
+  const bool lo_staged = a.split && lo_kind == 2;
+  auto put = [&](int64_t irow, int64_t icol, float v) {  // iterate element (irow, icol)
+    const int64_t xo = irow * ldc + icol;
     if (a.split) {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
       xb[xo] = h;
-      xl[xo] = __float2bfloat16_rn(v - __bfloat162float(h));
+      if (!lo_staged)
+        xl[lo_index(lo_kind, gd.r, ldc, irow, icol)] = __float2bfloat16_rn(v - __bfloat162float(h));
     } else {
       xf[xo] = v;
     }
@@ -135,13 +141,13 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
             l.lo = __floats2bfloat162_rn(nv[0] - h01.x, nv[1] - h01.y);
             l.hi = __floats2bfloat162_rn(nv[2] - h23.x, nv[3] - h23.y);
             *reinterpret_cast<Bf16x4*>(xb + xo) = h;
-            *reinterpret_cast<Bf16x4*>(xl + xo) = l;
+            if (!lo_staged) *reinterpret_cast<Bf16x4*>(xl + lo_index(lo_kind, gd.r, ldc, row, col)) = l;
           } else {
             *reinterpret_cast<float4*>(xf + xo) = make_float4(nv[0], nv[1], nv[2], nv[3]);
           }
         }
       }
-      if (transposed) {
+      if (transposed || lo_staged) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) stage[rr][c4 + e] = nv[e];
       }
@@ -175,10 +181,10 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
         if (a.mode == 0) __stcs(md.M + off, mo);
         sumsq += nv * nv;
         if (!transposed) {
-          put(row * ldc + col, nv);
+          put(row, col, nv);
         }
       }
-      if (transposed) stage[rr][cc] = nv;
+      if (transposed || lo_staged) stage[rr][cc] = nv;
     }
   }
 
@@ -201,13 +207,55 @@ __global__ void __launch_bounds__(256) ew_kernel(const __grid_constant__ EwArgs 
           const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
           const float2 fh = __bfloat1622float2(h);
           *reinterpret_cast<__nv_bfloat162*>(xb + xo) = h;
-          *reinterpret_cast<__nv_bfloat162*>(xl + xo) = __floats2bfloat162_rn(v0 - fh.x, v1 - fh.y);
+          if (!lo_staged)
+            *reinterpret_cast<__nv_bfloat162*>(xl + lo_index(lo_kind, gd.r, ldc, j, i)) =
+                __floats2bfloat162_rn(v0 - fh.x, v1 - fh.y);
         } else {
           *reinterpret_cast<float2*>(xf + xo) = make_float2(v0, v1);
         }
       } else {
-        put(xo, v0);
+        put(j, i, v0);
       }
+    }
+  }
+
+  if (lo_staged) {
+    // low part of a mid-size matrix, [col / 8][row][col % 8]: 16-byte pieces,
+    // consecutive threads on consecutive iterate rows (contiguous addresses)
+    if (!transposed) __syncthreads();  // (the transposed pass has synchronised already)
+    constexpr int kPieces = kEwRows * kEwCols / 8;
+    for (int p = tid; p < kPieces; p += blockDim.x) {
+      float v[8];
+      int64_t irow, icol0;
+      if (!transposed) {
+        // iterate rows = caller rows row0 .., columns col0 + 8 g ..
+        const int g = p / kEwRows, rr = p % kEwRows;
+        irow = row0 + rr;
+        icol0 = col0 + 8 * g;
+        if (irow >= n || icol0 >= m) continue;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = stage[rr][8 * g + e];
+      } else {
+        // iterate rows = caller columns col0 + cc, columns = caller rows row0 + 8 g ..
+        const int g = p / kEwCols, cc = p % kEwCols;
+        irow = col0 + cc;
+        icol0 = row0 + 8 * g;
+        if (irow >= m || icol0 >= n) continue;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = stage[8 * g + e][cc];
+      }
+      Bf16x4 l0, l1;
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]), h3 = __floats2bfloat162_rn(v[6], v[7]);
+      const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+      const float2 f2 = __bfloat1622float2(h2), f3 = __bfloat1622float2(h3);
+      l0.lo = __floats2bfloat162_rn(v[0] - f0.x, v[1] - f0.y);
+      l0.hi = __floats2bfloat162_rn(v[2] - f1.x, v[3] - f1.y);
+      l1.lo = __floats2bfloat162_rn(v[4] - f2.x, v[5] - f2.y);
+      l1.hi = __floats2bfloat162_rn(v[6] - f3.x, v[7] - f3.y);
+      __nv_bfloat16* dst = xl + lo_index(lo_kind, gd.r, ldc, irow, icol0);  // 16-byte aligned
+      reinterpret_cast<Bf16x4*>(dst)[0] = l0;
+      reinterpret_cast<Bf16x4*>(dst)[1] = l1;
     }
   }
 

@@ -23,6 +23,10 @@ cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, boo
 // per matrix (bf16 precision).
 cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream);
 
+// The same for min(n, m) <= 128 < max(n, m) <= 512, one 512-thread CTA per
+// matrix (args.small_mats lists those matrices).
+cudaError_t launch_mid(const SmallArgs& args, int grid, cudaStream_t stream);
+
 // Unit-RMS update scale, grouped / fp32 path: per-matrix RMS of O' from the
 // last Apply's sums of squares, then W <- W (1 - lr wd) - lr (gamma / RMS) O'.
 cudaError_t launch_rms_reduce(const FinishArgs& args, cudaStream_t stream);

@@ -24,6 +24,9 @@ constexpr int kBK = 64;
 // Matrices with min(n, m) <= kSmallMax and max(n, m) <= kSmallMax run the
 // whole Newton-Schulz iteration in one CTA (bf16 precision).
 constexpr int kSmallMax = 128;
+// Matrices with min(n, m) <= kSmallMax < max(n, m) <= kMidMaxC run the whole
+// iteration in one 512-thread CTA with the iterate in shared memory.
+constexpr int kMidMaxC = 512;
 
 // fp32 validation tile shape.
 constexpr int kSBM = 64;
@@ -65,7 +68,7 @@ struct GroupDesc {
   int32_t ldc, ldr;      // leading dimensions (elements) of r x c and r x r buffers
   int32_t count;         // matrices in this group
   int32_t first_mat;     // internal index of the group's first matrix
-  int32_t small;         // 1: runs in the small-matrix kernel, no stage tiles
+  int32_t small;         // 1: small-matrix kernel, 2: mid-size kernel (no stage tiles either way)
   int32_t pad0;
   int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate, ping-pong (fp32 mode)
   int64_t xb_off[2];     // bf16 iterate (bf16 mode: its high part, the MMA operand), ping-pong
@@ -171,6 +174,16 @@ struct FinishArgs {
   float lr, wd, gamma;
   float* diag;              // optional: diag[2 caller + 1] = RMS of the applied update O
 };
+
+// Element offset of iterate element (row, col) in a matrix's bf16 low-part
+// buffer (r x ldc elements). Row-major, except for the mid-size kernel's
+// matrices (GroupDesc.small == 2), whose low part is stored as 8-column
+// groups, [col / 8][row][col % 8], so that the threads that own consecutive
+// rows read and write one contiguous 16-byte piece each.
+__host__ __device__ __forceinline__ int64_t lo_index(int small, int r, int64_t ldc, int64_t row,
+                                                     int64_t col) {
+  return small == 2 ? ((col >> 3) * r + row) * 8 + (col & 7) : row * ldc + col;
+}
 
 // error bits in the device error word
 enum ErrBits : int { kErrTimeout = 1, kErrBadTile = 2 };

@@ -134,13 +134,15 @@ def expected_workspace(shapes, prec):
     off = al(off + ew * 4, 256)     # matrix of each elementwise tile
     small = [(n, m) for n, m in shapes if prec == MUON_NS_BF16 and max(n, m) <= 128]
     off = al(off + len(small) * 4, 256)  # small-matrix list
+    mid = [(n, m) for n, m in shapes if prec == MUON_NS_BF16 and min(n, m) <= 128 < max(n, m) <= 512]
+    off = al(off + len(mid) * 4, 256)  # mid-size list
     off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
     # unit-RMS scale: sums of squares per Apply tile (16 slots on tensor cores), a factor per matrix
     if prec == MUON_NS_BF16:
         apply_tiles = sum(len(mem) * math.ceil(r / 256) * math.ceil(c / 256)
-                          for (r, c), mem in groups.items() if c > 128)
+                          for (r, c), mem in groups.items() if r > 128 or c > 512)
         slots = 16
     else:
         apply_tiles = sum(len(mem) * math.ceil(r / 64) * math.ceil(c / 64) for (r, c), mem in groups.items())
@@ -164,7 +166,7 @@ def expected_workspace(shapes, prec):
 
 @pytest.mark.parametrize("prec", [MUON_NS_BF16, MUON_NS_FP32])
 def test_workspace_size_matches_layout(lib, prec):
-    shapes = [(256, 512), (512, 256), (7, 3), (1000, 130), (130, 1000), (1, 1)]
+    shapes = [(256, 512), (512, 256), (7, 3), (1000, 130), (130, 1000), (1, 1), (100, 300), (300, 100)]
     shapes += [(k, 2 * k + 1) for k in range(2, 40)]  # many groups: descriptor bytes matter
     st, plan = create(lib, shapes, prec)
     assert st == MUON_OK
@@ -193,8 +195,13 @@ def test_launch_list(lib):
     assert launch_list(lib, [(64, 64)]) == [0, 5]
     assert launch_list(lib, [(128, 128), (1, 1), (7, 100)]) == [0, 5]
     assert launch_list(lib, [(300, 400)]) == [0] + grouped
-    assert launch_list(lib, [(129, 64)]) == [0] + grouped
+    # min(n, m) <= 128 < max(n, m) <= 512: the one-CTA mid-size kernel (kind 8)
+    assert launch_list(lib, [(129, 64)]) == [0, 8]
+    assert launch_list(lib, [(128, 512), (512, 100), (1, 129)]) == [0, 8]
+    assert launch_list(lib, [(128, 513)]) == [0] + grouped
+    assert launch_list(lib, [(129, 129)]) == [0] + grouped
     assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 5] + grouped
+    assert launch_list(lib, [(64, 64), (100, 300), (300, 400)]) == [0, 5, 8] + grouped
     # the fp32 validation precision has no small-matrix kernel
     assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + grouped
 

@@ -314,3 +314,34 @@ def test_l2_batching_gives_identical_results(precision):
     assert ms.sync_status() == 0
     for k in range(a.count):
         assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k]) and torch.equal(Oa[k], Ob[k])
+
+
+MID = [(128, 512), (512, 128), (100, 300), (300, 100), (1, 200), (128, 129), (64, 512),
+       (77, 333), (129, 64)]
+
+
+@pytest.mark.parametrize("spectrum", ["geometric", "flat"])
+def test_mid_size_kernel(spectrum):
+    """min(n, m) <= 128 < max(n, m) <= 512: the one-CTA mid-size kernel, both
+    orientations, ragged edges, a single row, several steps."""
+    wl = workloads.make_random(MID, device="cuda", seed=43, spectrum=spectrum)
+    worst = check_step(wl, "bf16", steps=2)
+    assert worst["O_over_tol"] <= 1.0, worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+@pytest.mark.parametrize("scale_mode", ["unit_rms", "none"])
+def test_mid_size_kernel_scale_modes(scale_mode):
+    wl = workloads.make_random(MID[:4], device="cuda", seed=47)
+    hyper = dict(wl.hyper, gamma=0.2 if scale_mode == "unit_rms" else 1.0)
+    worst = check_step(wl, "bf16", hyper=hyper, scale_mode=scale_mode)
+    assert worst["O_over_tol"] <= 1.0, worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+def test_mid_size_kernel_orthogonalize():
+    """ns_orthogonalize through the mid-size kernel (no weight update)."""
+    rng = torch.Generator(device="cuda").manual_seed(5)
+    xs = [torch.randn(n, m, generator=rng, device="cuda") for n, m in MID]
+    errs = check_ns(xs, "bf16")
+    assert all_within(errs), errs
