@@ -489,7 +489,8 @@ def main():
                "sample": f"{done} of {wl.count} matrices of {args.config}, {dt:.1f} s of float64 numpy"}
 
     if rank == 0:
-        names = {0: "elementwise", 1: "gram", 2: "poly", 3: "apply", 4: "apply_update", 5: "small"}
+        names = {0: "elementwise", 1: "gram", 2: "poly", 3: "apply", 4: "apply_update", 5: "small",
+                 6: "rms_reduce", 7: "update", 8: "mid"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

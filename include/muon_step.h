@@ -172,7 +172,9 @@ MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* h
 /* Number of kernel launches one execute issues, and the kind of each
  * (0 momentum/norm/cast, 1 Gram, 2 polynomial, 3 apply, 4 apply + update,
  * 5 small-matrix kernel (all steps and the update of matrices up to
- * 128 x 128), 6 per-matrix RMS reduction, 7 update pass). */
+ * 128 x 128), 6 per-matrix RMS reduction, 7 update pass, 8 mid-size kernel
+ * (all steps and the update of matrices with min(n, m) <= 128 < max(n, m)
+ * <= 512)). */
 MUON_API muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds);
 
 /* Optional timing: `events` holds 2 * launches cudaEvent_t (as void*); each
