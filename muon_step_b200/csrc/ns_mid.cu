@@ -89,6 +89,13 @@ __device__ __forceinline__ void gemm_apply(uint32_t d, uint32_t sb, uint32_t sx,
   }
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Write 32 values of row i, columns 32 ch .., as bf16 into a swizzled tile.
 __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const float (&v)[32]) {
 #pragma unroll
@@ -238,9 +245,19 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
         gemm_apply(tmem, sB, sX, nh);
         ptx::umma_commit(bar_mma);
       }
+      const bool last = (k + 1 == a.steps);
+      // while the product runs: this thread's low-part pieces into L1, and on
+      // the last step the caller's weight into L2 for the update
+      if (row_in) {
+        for (int g = 16 * cq; g < 16 * cq + 16 && 8 * g < c; ++g)
+          prefetch_l1(xl + static_cast<int64_t>(g) * r * 8);
+      }
+      if (last && md.W) {
+        const int64_t lines = (md.n * md.m + 31) / 32;  // 128-byte lines of W
+        for (int64_t ln = tid; ln < lines; ln += kThreads) prefetch_l2(md.W + ln * 32);
+      }
       wait_mma();
       if (!ok) break;
-      const bool last = (k + 1 == a.steps);
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         const int col0 = 128 * cq + 32 * j;
@@ -335,43 +352,63 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
       __syncthreads();
       if (!tr) {
         // caller rows = iterate rows (r), caller columns p0 .. p0 + bw
-        for (int crow = warp; crow < r; crow += kThreads / 32) {
-          float* Wr = md.W ? md.W + static_cast<int64_t>(crow) * md.m + p0 : nullptr;
-          float* Or = md.O ? md.O + static_cast<int64_t>(crow) * md.m + p0 : nullptr;
-          float w[4], o[4];
+        // two caller rows per warp pass: all loads before the stores
+        for (int cb = 2 * warp; cb < r; cb += 2 * (kThreads / 32)) {
+          float w[2][4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int lc = 32 * q + lane;
-            o[q] = T[crow * 128 + (lc ^ (crow & 31))];
-            w[q] = (lc < bw && Wr) ? Wr[lc] : 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const int crow = cb + u;
+            float* Wr = (md.W && crow < r) ? md.W + static_cast<int64_t>(crow) * md.m + p0 : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int lc = 32 * q + lane;
+              w[u][q] = (lc < bw && Wr) ? Wr[lc] : 0.f;
+            }
           }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int lc = 32 * q + lane;
-            if (lc >= bw) continue;
-            if (Or) Or[lc] = o[q];
-            if (Wr) Wr[lc] = fmaf(w[q], uc.keep, -uc.step * o[q]);
+          for (int u = 0; u < 2; ++u) {
+            const int crow = cb + u;
+            if (crow >= r) break;
+            float* Wr = md.W ? md.W + static_cast<int64_t>(crow) * md.m + p0 : nullptr;
+            float* Or = md.O ? md.O + static_cast<int64_t>(crow) * md.m + p0 : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int lc = 32 * q + lane;
+              if (lc >= bw) continue;
+              const float o = T[crow * 128 + (lc ^ (crow & 31))];
+              if (Or) Or[lc] = o;
+              if (Wr) Wr[lc] = fmaf(w[u][q], uc.keep, -uc.step * o);
+            }
           }
         }
       } else {
         // caller rows p0 .. p0 + bw = iterate columns, caller columns = iterate rows (r)
-        for (int cr = warp; cr < bw; cr += kThreads / 32) {
-          const int64_t crow = p0 + cr;
-          float* Wr = md.W ? md.W + crow * md.m : nullptr;
-          float* Or = md.O ? md.O + crow * md.m : nullptr;
-          float w[4], o[4];
+        for (int cb = 2 * warp; cb < bw; cb += 2 * (kThreads / 32)) {
+          float w[2][4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = 32 * q + lane;  // iterate row
-            o[q] = T[col * 128 + (cr ^ (col & 31))];
-            w[q] = (col < r && Wr) ? Wr[col] : 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const int cr = cb + u;
+            float* Wr = (md.W && cr < bw) ? md.W + (p0 + cr) * md.m : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = 32 * q + lane;  // iterate row
+              w[u][q] = (col < r && Wr) ? Wr[col] : 0.f;
+            }
           }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = 32 * q + lane;
-            if (col >= r) continue;
-            if (Or) Or[col] = o[q];
-            if (Wr) Wr[col] = fmaf(w[q], uc.keep, -uc.step * o[q]);
+          for (int u = 0; u < 2; ++u) {
+            const int cr = cb + u;
+            if (cr >= bw) break;
+            float* Wr = md.W ? md.W + (p0 + cr) * md.m : nullptr;
+            float* Or = md.O ? md.O + (p0 + cr) * md.m : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = 32 * q + lane;
+              if (col >= r) continue;
+              const float o = T[col * 128 + (cr ^ (col & 31))];
+              if (Or) Or[col] = o;
+              if (Wr) Wr[col] = fmaf(w[u][q], uc.keep, -uc.step * o);
+            }
           }
         }
       }
