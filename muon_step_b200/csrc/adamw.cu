@@ -5,12 +5,13 @@
 // 输出头、bias、RMSNorm 还在用 AdamW" (which parameters stay on AdamW);
 // Algorithm 1 step five (decoupled decay as a factor 1 - lr wd).
 //
-// Layout: every tensor is cut into chunks of kChunk elements; one CTA of 256
-// threads takes one chunk, each thread 4 groups of 4 consecutive elements at
-// stride 1024, so that every warp access is one contiguous 512-byte segment.
-// Each thread issues all 16 of its 16-byte loads (p, g, m, v) before the first
-// store. The chunk -> tensor map is a binary search over the tensors' first
-// chunk indices (a few cached loads per CTA). HBM-bound: 28 bytes per element.
+// Layout: a host-built work list gives each CTA of 256 threads one item:
+// either a 4096-element chunk of a large tensor (each thread 4 groups of 4
+// consecutive elements at stride 1024, every warp access one contiguous
+// 512-byte segment, all 16 of a thread's 16-byte loads issued before its
+// first store), or a bundle of consecutive small tensors (up to 4096
+// elements in all), one tensor per warp at a time, so that thousands of bias
+// and norm vectors do not each occupy a CTA. HBM-bound: 28 bytes per element.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -38,15 +39,22 @@ struct AdamwTensor {
   float* m;
   float* v;
   int64_t numel;
-  int64_t chunk_begin;  // first chunk of this tensor
   int32_t vec;          // all four pointers 16-byte aligned
   int32_t pad;
 };
 
+// One CTA's work: chunk `chunk` of tensor `first`, or (chunk < 0) every
+// element of tensors first .. last - 1.
+struct AdamwWork {
+  int32_t first, last;
+  int64_t chunk;
+};
+
 struct AdamwArgs {
   const AdamwTensor* tensors;
+  const AdamwWork* work;
   int32_t count;
-  int64_t total_chunks;
+  int64_t total_chunks;  // work items
   float beta1, beta2, one_minus_b1, one_minus_b2, eps, keep;
   float step_size;      // lr / (1 - beta1^t)
   float inv_sqrt_bc2;   // 1 / sqrt(1 - beta2^t)
@@ -71,17 +79,9 @@ __device__ __forceinline__ void adamw_elem(const AdamwArgs& a, const Consts& k, 
 }
 
 __global__ void __launch_bounds__(kThreads) adamw_kernel(const __grid_constant__ AdamwArgs a) {
-  __shared__ int tensor_s;
   __shared__ Consts consts_s;
-  const int64_t chunk = blockIdx.x;
+  const AdamwWork wk = a.work[blockIdx.x];
   if (threadIdx.x == 0) {
-    int lo = 0, hi = a.count - 1;  // last tensor with chunk_begin <= chunk
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(&a.tensors[mid].chunk_begin) <= chunk) lo = mid;
-      else hi = mid - 1;
-    }
-    tensor_s = lo;
     Consts k{a.step_size, a.inv_sqrt_bc2};
     if (a.step_dev) {
       const int t = max(1, *a.step_dev);
@@ -93,10 +93,30 @@ __global__ void __launch_bounds__(kThreads) adamw_kernel(const __grid_constant__
     consts_s = k;
   }
   __syncthreads();
-  const AdamwTensor T = a.tensors[tensor_s];
   const Consts k = consts_s;
-  const int64_t base = (chunk - T.chunk_begin) * kChunk;
   const int tid = threadIdx.x;
+  if (wk.chunk < 0) {
+    // bundle of small tensors: one per warp at a time
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int t = wk.first + warp; t < wk.last; t += kThreads / 32) {
+      float* tp = a.tensors[t].p;
+      const float* tg = a.tensors[t].g;
+      float* tm = a.tensors[t].m;
+      float* tv = a.tensors[t].v;
+      const int64_t numel = a.tensors[t].numel;
+      // small tensors: element per lane, each warp access 128 contiguous bytes
+      for (int64_t e = lane; e < numel; e += 32) {
+        float p = tp[e], m = tm[e], v = tv[e];
+        adamw_elem(a, k, p, tg[e], m, v);
+        tp[e] = p;
+        tm[e] = m;
+        tv[e] = v;
+      }
+    }
+    return;
+  }
+  const AdamwTensor T = a.tensors[wk.first];
+  const int64_t base = wk.chunk * kChunk;
   if (T.vec && base + kChunk <= T.numel) {
     float4 p[kGroups], g[kGroups], m[kGroups], v[kGroups];
 #pragma unroll
@@ -144,6 +164,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 struct muon_adamw_plan_s {
   std::vector<muon::AdamwTensor> tensors;
+  std::vector<muon::AdamwWork> work;
+  size_t off_work = 0;
   int64_t total_chunks = 0;
   int64_t numel = 0;
   size_t ws_bytes = 0;
@@ -181,7 +203,6 @@ muon_status_t muon_adamw_plan_create(const muon_adamw_param_t* params, int count
     t.m = q.m;
     t.v = q.v;
     t.numel = q.numel;
-    t.chunk_begin = chunks;
     t.vec = aligned16(q.p) && aligned16(q.g) && aligned16(q.m) && aligned16(q.v);
     chunks += (q.numel + kChunk - 1) / kChunk;
     p->numel += q.numel;
@@ -191,8 +212,36 @@ muon_status_t muon_adamw_plan_create(const muon_adamw_param_t* params, int count
     delete p;
     return MUON_ERR_UNSUPPORTED;
   }
-  p->total_chunks = chunks;
-  p->ws_bytes = align_up(std::max<size_t>(p->tensors.size(), 1) * sizeof(AdamwTensor), 256);
+  // work list: chunks of tensors above half a chunk; runs of smaller ones in
+  // bundles of at most kChunk elements (and 64 tensors)
+  const int nt = static_cast<int>(p->tensors.size());
+  int b0 = -1;
+  int64_t bsum = 0;
+  auto flush = [&](int end) {
+    if (b0 >= 0) p->work.push_back(AdamwWork{b0, end, -1});
+    b0 = -1;
+    bsum = 0;
+  };
+  for (int t = 0; t < nt; ++t) {
+    const int64_t n = p->tensors[t].numel;
+    if (n > kChunk / 2) {
+      flush(t);
+      const int64_t nc = (n + kChunk - 1) / kChunk;
+      for (int64_t ch = 0; ch < nc; ++ch) p->work.push_back(AdamwWork{t, t + 1, ch});
+      continue;
+    }
+    if (b0 >= 0 && (bsum + n > kChunk || t - b0 >= 64)) flush(t);
+    if (b0 < 0) b0 = t;
+    bsum += n;
+  }
+  flush(nt);
+  if (static_cast<int64_t>(p->work.size()) > 0x7fffffffLL) {
+    delete p;
+    return MUON_ERR_UNSUPPORTED;
+  }
+  p->total_chunks = static_cast<int64_t>(p->work.size());
+  p->off_work = align_up(std::max<size_t>(p->tensors.size(), 1) * sizeof(AdamwTensor), 256);
+  p->ws_bytes = p->off_work + align_up(std::max<size_t>(p->work.size(), 1) * sizeof(AdamwWork), 256);
   *plan = p;
   return MUON_OK;
 }
@@ -229,13 +278,17 @@ muon_status_t muon_adamw_plan_execute(muon_adamw_plan_t plan, const muon_adamw_h
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   if (workspace != plan->uploaded_ws || dev != plan->uploaded_dev) {
     if (cudaMemcpyAsync(workspace, plan->tensors.data(), plan->tensors.size() * sizeof(AdamwTensor),
-                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<char*>(workspace) + plan->off_work, plan->work.data(),
+                        plan->work.size() * sizeof(AdamwWork), cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
       return MUON_ERR_CUDA;
     plan->uploaded_ws = workspace;
     plan->uploaded_dev = dev;
   }
   AdamwArgs a{};
   a.tensors = static_cast<const AdamwTensor*>(workspace);
+  a.work = reinterpret_cast<const AdamwWork*>(static_cast<const char*>(workspace) + plan->off_work);
   a.count = static_cast<int32_t>(plan->tensors.size());
   a.total_chunks = plan->total_chunks;
   const double b1 = h->beta1, b2 = h->beta2;

@@ -64,14 +64,36 @@ def test_plan_validation(lib):
     lib.muon_adamw_plan_destroy(plan)
 
 
-@pytest.mark.parametrize("sizes", [[1], [4096, 4097, 3], [0, 0, 1, 2, 3, 4, 5, 6]])
-def test_workspace_holds_one_entry_per_nonempty_tensor(lib, sizes):
+def work_items(sizes, chunk=4096):
+    """The work list rule: 4096-element chunks of tensors above 2048 elements;
+    runs of smaller tensors in bundles of at most 4096 elements and 64 tensors."""
+    items, start, total, count = 0, None, 0, 0
+    for n in (s for s in sizes if s > 0):
+        if n > chunk // 2:
+            items += (start is not None) + -(-n // chunk)
+            start, total, count = None, 0, 0
+            continue
+        if start is not None and (total + n > chunk or count >= 64):
+            items += 1
+            start, total, count = None, 0, 0
+        if start is None:
+            start = True
+        total += n
+        count += 1
+    return items + (start is not None)
+
+
+@pytest.mark.parametrize("sizes", [[1], [4096, 4097, 3], [0, 0, 1, 2, 3, 4, 5, 6],
+                                   [128] * 200, [100, 5000, 100, 100, 3000, 2000] * 3])
+def test_workspace_holds_the_tensor_table_and_the_work_list(lib, sizes):
     st, plan = create(lib, adamw_params(sizes))
     assert st == MUON_OK
     ws = ctypes.c_size_t()
     assert lib.muon_adamw_plan_workspace_size(plan, ctypes.byref(ws)) == MUON_OK
     nonempty = sum(1 for n in sizes if n > 0)
-    assert ws.value == (nonempty * 48 + 255) // 256 * 256  # 48-byte table entries
+    al = lambda x: (x + 255) // 256 * 256
+    # 48-byte tensor entries, then 16-byte work items
+    assert ws.value == al(max(nonempty, 1) * 48) + al(max(work_items(sizes), 1) * 16)
     one = ctypes.c_size_t()
     assert lib.muon_adamw_workspace_size(adamw_params(sizes), len(sizes), ctypes.byref(one)) == MUON_OK
     assert one.value == ws.value
@@ -236,3 +258,31 @@ def test_hybrid_optimizer_end_to_end():
             assert _rel(got, ref[n]) <= TOL, n
     assert torch.isfinite(diag).all()
     assert (diag[:, 1] > 0.15).all() and (diag[:, 1] < 0.25).all(), diag
+
+
+@pytest.mark.gpu
+def test_many_small_tensors_in_bundles():
+    """Hundreds of bias / norm sized tensors (bundled several per CTA) mixed
+    with large ones, against the oracle."""
+    import muon_step_b200 as ms
+    from oracle import companion_oracle as co
+
+    rng = np.random.default_rng(9)
+    sizes = [int(s) for s in rng.integers(1, 3000, 300)] + [70000, 5, 9000]
+    state = _tensors(sizes, seed=11, unaligned=(3, 150, 301))
+    gen = torch.Generator(device="cuda").manual_seed(12)
+    grads = [torch.randn(s[0].shape, generator=gen, device="cuda") * 1e-2 for s in state]
+    ref = [[s[0].double().cpu().numpy(), s[1].double().cpu().numpy(), s[2].double().cpu().numpy()]
+           for s in state]
+    plan = ms.AdamWPlan([(p, g, m, v) for (p, m, v), g in zip(state, grads)])
+    ws = plan.alloc_workspace()
+    for t in (1, 2):
+        plan.execute(ws, step=t)
+        for k, g in enumerate(grads):
+            ref[k] = list(co.adamw_step(ref[k][0], g.double().cpu().numpy(), ref[k][1], ref[k][2], t,
+                                        lr=0.02, wd=0.1))
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for k, (p, m, v) in enumerate(state):
+        for got, want in ((p, ref[k][0]), (m, ref[k][1]), (v, ref[k][2])):
+            assert _rel(got.double().cpu().numpy(), want) <= TOL, sizes[k]
