@@ -200,7 +200,8 @@ def test_distributed_step_world_one_matches_plan():
 def test_scale_modes(precision, scale_mode):
     """Unit-RMS and no-rescale updates on small, large, transposed and
     unaligned matrices (small-matrix kernel, grouped kernels, update pass)."""
-    shapes = [(64, 64), (100, 37), (300, 520), (520, 300), (257, 129), (1, 7)]
+    shapes = [(64, 64), (100, 37), (300, 520), (520, 300), (257, 129), (1, 7), (40, 1024),
+              (130, 2048)]
     wl = workloads.make_random(shapes, device="cuda", seed=29)
     hyper = dict(wl.hyper, gamma=0.2 if scale_mode == "unit_rms" else 1.0)
     worst = check_step(wl, precision, hyper=hyper, scale_mode=scale_mode)
