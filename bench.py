@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
+    ap.add_argument("--count", type=int, default=None,
+                    help="sweep workloads only: this many matrices instead of ~16 GB of state "
+                         "(small cases for profiling; not a benchmark line)")
     return ap.parse_args()
 
 
@@ -326,7 +329,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    wl = workloads.make(args.config, device=dev)
+    if args.count is not None and not args.config.startswith("sweep_"):
+        raise SystemExit("--count applies to the sweep workloads only")
+    wl = workloads.make(args.config, device=dev,
+                        **({"count": args.count} if args.count is not None else {}))
     h = wl.hyper
     params = [(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)]
     plan = ms.MuonPlan(params, precision=args.precision)
