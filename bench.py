@@ -423,12 +423,17 @@ def main():
         dom_name = "stage_tc_kernel<Apply>" if args.precision == "bf16" else "stage_simt_kernel<Apply>"
         traffic = traffic_from_profile(args.config)
     else:
-        # every matrix runs in the small-matrix kernel: all steps in one launch;
-        # bytes: fp32 + bf16 iterate read, W read and written (14 B per element)
-        dom_flops = g_fl + p_fl + a_fl
-        dom_bytes = sum(14.0 * n * m for n, m in wl.shapes)
-        dom_ms = avg[5]
-        dom_name = "ns_small_kernel"
+        # every matrix runs in the one-CTA kernels (all steps in one launch):
+        # the small-matrix (5) or the mid-size (8) kernel, whichever took longer;
+        # bytes: iterate high + low parts read, W read and written (12 B per element)
+        kd = max((k for k in (5, 8) if k in share), key=lambda k: share[k])
+        mine = [(n, m) for n, m in wl.shapes
+                if (max(n, m) <= 128) == (kd == 5) and min(n, m) <= 128 and max(n, m) <= 512]
+        dom_flops = sum(ns_steps * (4.0 * min(n, m) ** 2 * max(n, m) + 2.0 * min(n, m) ** 3)
+                        for n, m in mine)
+        dom_bytes = sum(12.0 * n * m for n, m in mine)
+        dom_ms = avg[kd]
+        dom_name = "ns_small_kernel" if kd == 5 else "ns_mid_kernel"
         traffic = None
     t_tensor = dom_flops / (tensor_peak * 1e12)
     t_hbm = dom_bytes / (hbm_peak * 1e9)
