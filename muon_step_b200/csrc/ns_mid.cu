@@ -107,6 +107,67 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const fl
   }
 }
 
+// One 32-column chunk of the Apply epilogue for iterate row `row`:
+// X' = alpha (a X + v) with X = high (shared) + low (global), written back as
+// high and low parts. kFirst folds alpha (step one), kLast accumulates the
+// sum of squares, kMask zeroes what lies outside the matrix (ragged chunks).
+template <bool kFirst, bool kLast, bool kMask>
+__device__ __forceinline__ void apply_chunk(uint8_t* Xs, __nv_bfloat16* xl, int row, int col0, int r,
+                                            int c, bool row_in, float alpha, float ca,
+                                            const float (&v)[32], float& ssq) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int p = col0 / 8 + q;
+    Bf16x8 h8 = *reinterpret_cast<const Bf16x8*>(Xs + piece_off(row, p));
+    const bool grp = !kMask || (row_in && col0 + 8 * q < c);  // 8 columns that start inside
+    __nv_bfloat16* lp = xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8;
+    uint4 lraw = make_uint4(0u, 0u, 0u, 0u);
+    if (grp) lraw = *reinterpret_cast<const uint4*>(lp);
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lraw);
+    Bf16x8 lo8;
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      const int e = 8 * q + 2 * hh;
+      const float2 fh = __bfloat1622float2(h8.v[hh]);
+      const float2 fl = __bfloat1622float2(l2[hh]);
+      float x0 = fh.x + fl.x, x1 = fh.y + fl.y;
+      if (kMask) {
+        // columns c .. ldc of the low part are not written by the elementwise kernel
+        x0 = (row_in && col0 + e < c) ? x0 : 0.f;
+        x1 = (row_in && col0 + e + 1 < c) ? x1 : 0.f;
+      }
+      float y0 = fmaf(ca, x0, v[e]), y1 = fmaf(ca, x1, v[e + 1]);
+      if (kFirst) {
+        y0 *= alpha;
+        y1 *= alpha;
+      }
+      if (kLast) ssq = fmaf(y0, y0, fmaf(y1, y1, ssq));
+      h8.v[hh] = __floats2bfloat162_rn(y0, y1);
+      const float2 nh2 = __bfloat1622float2(h8.v[hh]);
+      lo8.v[hh] = __floats2bfloat162_rn(y0 - nh2.x, y1 - nh2.y);
+    }
+    *reinterpret_cast<Bf16x8*>(Xs + piece_off(row, p)) = h8;
+    if (grp) *reinterpret_cast<Bf16x8*>(lp) = lo8;
+  }
+}
+
+template <bool kFirst, bool kLast>
+__device__ __forceinline__ void apply_epilogue(uint8_t* Xs, __nv_bfloat16* xl, uint32_t trow, int row,
+                                               int cq, int r, int c, bool row_in, float alpha,
+                                               float ca, float& ssq) {
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    const int col0 = 128 * cq + 32 * j;
+    if (col0 >= c) break;  // the same for the whole warp
+    float v[32];
+    ptx::tmem_ld32(trow + col0, v);
+    if (row_in && col0 + 32 <= c)
+      apply_chunk<kFirst, kLast, false>(Xs, xl, row, col0, r, c, row_in, alpha, ca, v, ssq);
+    else
+      apply_chunk<kFirst, kLast, true>(Xs, xl, row, col0, r, c, row_in, alpha, ca, v, ssq);
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_constant__ SmallArgs a) {
@@ -258,39 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
       }
       wait_mma();
       if (!ok) break;
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        const int col0 = 128 * cq + 32 * j;
-        if (col0 >= c) break;  // the same for the whole warp
-        float v[32];
-        ptx::tmem_ld32(trow + col0, v);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int p = col0 / 8 + q;
-          Bf16x8 h8 = *reinterpret_cast<const Bf16x8*>(Xs + piece_off(row, p));
-          const bool grp = row_in && col0 + 8 * q < c;  // 8 columns that start inside the matrix
-          uint4 lraw = make_uint4(0u, 0u, 0u, 0u);
-          if (grp) lraw = *reinterpret_cast<const uint4*>(xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8);
-          const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lraw);
-          Bf16x8 lo8;
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            const int e = 8 * q + 2 * hh;
-            const float2 fh = __bfloat1622float2(h8.v[hh]);
-            const float2 fl = __bfloat1622float2(l2[hh]);
-            // columns c .. ldc of the low part are not written by the elementwise kernel
-            const float x0 = (row_in && col0 + e < c) ? fh.x + fl.x : 0.f;
-            const float x1 = (row_in && col0 + e + 1 < c) ? fh.y + fl.y : 0.f;
-            const float y0 = alpha * fmaf(ca, x0, v[e]);
-            const float y1 = alpha * fmaf(ca, x1, v[e + 1]);
-            if (last) ssq = fmaf(y0, y0, fmaf(y1, y1, ssq));
-            h8.v[hh] = __floats2bfloat162_rn(y0, y1);
-            const float2 nh2 = __bfloat1622float2(h8.v[hh]);
-            lo8.v[hh] = __floats2bfloat162_rn(y0 - nh2.x, y1 - nh2.y);
-          }
-          *reinterpret_cast<Bf16x8*>(Xs + piece_off(row, p)) = h8;
-          if (grp) *reinterpret_cast<Bf16x8*>(xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8) = lo8;
-        }
+      // variants without the step-one scale, sums or masks where they are not needed
+      if (k == 0) {
+        if (last) apply_epilogue<true, true>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
+        else apply_epilogue<true, false>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
+      } else {
+        if (last) apply_epilogue<false, true>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
+        else apply_epilogue<false, false>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
       }
       hand_over();
     }
