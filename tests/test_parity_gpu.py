@@ -346,3 +346,21 @@ def test_mid_size_kernel_orthogonalize():
     xs = [torch.randn(n, m, generator=rng, device="cuda") for n, m in MID]
     errs = check_ns(xs, "bf16")
     assert all_within(errs), errs
+
+
+def test_megatron_recipe_settings():
+    """The DeepSeek-V4-Flash Megatron-Bridge recipe's Muon keys (5-step
+    quintic, unit-RMS scale x 0.2, fp32 products) through the config mapper."""
+    from muon_step_b200.config import from_megatron
+
+    cfg = from_megatron(muon_momentum=0.95, muon_use_nesterov=True, muon_scale_mode="unit_rms_norm",
+                        muon_fp32_matmul_prec="highest", muon_num_ns_steps=5,
+                        muon_extra_scale_factor=0.2, muon_coefficient_type="quintic",
+                        max_lr=2.7e-4, weight_decay=0.1)
+    wl = workloads.make_random([(96, 160), (300, 200), (64, 64)], device="cuda", seed=53)
+    hyper = dict(wl.hyper, lr=cfg.lr, mu=cfg.momentum, wd=cfg.weight_decay, gamma=cfg.gamma,
+                 nesterov=cfg.nesterov)
+    worst = check_step(wl, cfg.precision, hyper=hyper, schedule=cfg.schedule,
+                       scale_mode=cfg.scale_mode)
+    assert worst["O_over_tol"] <= 1.0, worst
+    assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
