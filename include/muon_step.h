@@ -222,6 +222,11 @@ MUON_API const char* muon_status_string(muon_status_t status);
 
 MUON_API int muon_abi_version(void);
 
+/* NVTX ranges (host side) around each kernel launch of later executes,
+ * named by launch kind ("muon:gram", "muon:apply", ...), for profilers that
+ * collect NVTX; off (0) by default. Process-wide. */
+MUON_API void muon_set_tracing(int on);
+
 /* Bound, in nanoseconds, on every device-side spin-wait of later launches
  * (default 2e9). Values below 1000 are raised to 1000. */
 MUON_API void muon_set_wait_limit_ns(uint64_t ns);

@@ -409,6 +409,11 @@ def sync_status(stream=None) -> int:
     return _lib.load().muon_sync_status(_stream_ptr(stream))
 
 
+def set_tracing(on: bool = True):
+    """NVTX ranges around every kernel launch of later executes (off by default)."""
+    _lib.load().muon_set_tracing(1 if on else 0)
+
+
 def set_wait_limit_ns(ns: int):
     _lib.load().muon_set_wait_limit_ns(int(ns))
 

@@ -36,7 +36,7 @@ EXPORTS = (
     "muon_adamw_plan_numel", "muon_adamw_plan_destroy", "muon_adamw_workspace_size",
     "muon_adamw_step",
     "muon_shard_workspace_size", "muon_shard_momentum", "muon_shard_update",
-    "muon_plan_set_l2_batching",
+    "muon_plan_set_l2_batching", "muon_set_tracing",
 )
 
 
@@ -109,6 +109,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_plan_set_scale_mode": (st, [vp, ctypes.c_int]),
         "muon_plan_set_diagnostics": (st, [vp, vp]),
         "muon_plan_set_l2_batching": (st, [vp, ctypes.c_size_t]),
+        "muon_set_tracing": (None, [ctypes.c_int]),
         "muon_adamw_plan_create": (st, [P(AdamwParam), ctypes.c_int, P(vp)]),
         "muon_adamw_plan_workspace_size": (st, [vp, P(ctypes.c_size_t)]),
         "muon_adamw_plan_execute": (st, [vp, P(AdamwHyper), vp, ctypes.c_size_t, vp]),

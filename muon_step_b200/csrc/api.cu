@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -18,6 +19,8 @@
 #include <new>
 #include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "kernels.cuh"
 #include "muon_step.h"
@@ -459,7 +462,28 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
 // Timing events around launches. Under stream capture the record must become
 // an external event node of the graph, or its timestamp cannot be read after
 // a replay.
+std::atomic<int> g_tracing{0};
+
+// NVTX range names of the launch kinds (host-side ranges around each launch;
+// a profiler attached to the process shows them, otherwise they cost a call)
+const char* kind_name(int kind) {
+  static const char* names[] = {"muon:momentum+norm", "muon:gram", "muon:poly", "muon:apply",
+                                "muon:apply+update", "muon:small", "muon:rms", "muon:update",
+                                "muon:mid"};
+  return (kind >= 0 && kind < 9) ? names[kind] : "muon:?";
+}
+
+// Slots come in pairs around launch slot / 2: timing events (when set) and
+// NVTX ranges (when tracing is on).
 muon_status_t record(muon_plan_s* p, int slot, cudaStream_t stream) {
+  if (g_tracing.load(std::memory_order_relaxed)) {
+    if ((slot & 1) == 0) {
+      const int k = slot / 2;
+      nvtxRangePushA(kind_name(k < static_cast<int>(p->launch_kinds.size()) ? p->launch_kinds[k] : -1));
+    } else {
+      nvtxRangePop();
+    }
+  }
   if (p->events.empty()) return MUON_OK;
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MUON_ERR_CUDA;
@@ -760,6 +784,8 @@ muon_status_t muon_plan_set_scale_mode(muon_plan_t plan, muon_scale_mode_t mode)
   plan->events.clear();  // the launch list may have changed: timing must be set again
   return MUON_OK;
 }
+
+void muon_set_tracing(int on) { g_tracing.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes) {
   if (!plan) return MUON_ERR_INVALID_ARG;

@@ -364,3 +364,24 @@ def test_megatron_recipe_settings():
                        scale_mode=cfg.scale_mode)
     assert worst["O_over_tol"] <= 1.0, worst
     assert worst["M"] <= TOL_ELEMENTWISE and worst["W_given_O"] <= TOL_ELEMENTWISE, worst
+
+
+def test_tracing_does_not_change_results():
+    """NVTX ranges around the launches change nothing on the device."""
+    import muon_step_b200 as ms
+
+    shapes = [(300, 520), (64, 64), (100, 300)]
+    a = workloads.make_random(shapes, device="cuda", seed=59)
+    b = workloads.make_random(shapes, device="cuda", seed=59)
+    pa = ms.MuonPlan([(a.W[k], a.G[k], a.M[k]) for k in range(a.count)])
+    pb = ms.MuonPlan([(b.W[k], b.G[k], b.M[k]) for k in range(b.count)])
+    ms.set_tracing(True)
+    try:
+        pa.execute()
+    finally:
+        ms.set_tracing(False)
+    pb.execute()
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for k in range(a.count):
+        assert torch.equal(a.W[k], b.W[k]) and torch.equal(a.M[k], b.M[k])
