@@ -338,3 +338,35 @@ def test_l2_batching_repeats_the_stage_launches_per_batch(lib):
     assert lib.muon_plan_set_l2_batching(plan, 0) == MUON_OK
     assert kinds_now() == [0, 5] + one_pass
     lib.muon_plan_destroy(plan)
+
+
+try:
+    from hypothesis import given, settings
+    from hypothesis import strategies as hst
+except ImportError:  # pragma: no cover
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=60, deadline=None)
+    @given(hst.lists(hst.tuples(hst.integers(1, 3000), hst.integers(1, 3000)), min_size=1, max_size=12),
+           hst.sampled_from([MUON_NS_BF16, MUON_NS_FP32]))
+    def test_planner_layout_and_launches_for_random_shapes(shapes, prec):
+        """For any list of shapes the workspace follows the layout rule and the
+        launch list holds the elementwise pass, the one-CTA kernels the shapes
+        need and one pass of stage launches when a larger matrix is present."""
+        lib = _lib.load()
+        st, plan = create(lib, shapes, prec)
+        assert st == MUON_OK
+        n = ctypes.c_size_t()
+        assert lib.muon_plan_workspace_size(plan, ctypes.byref(n)) == MUON_OK
+        lib.muon_plan_destroy(plan)
+        assert n.value == expected_workspace(shapes, prec)
+        tc = prec == MUON_NS_BF16
+        small = tc and any(max(a, b) <= 128 for a, b in shapes)
+        mid = tc and any(min(a, b) <= 128 < max(a, b) <= 512 for a, b in shapes)
+        large = any(not tc or not (min(a, b) <= 128 and max(a, b) <= 512) for a, b in shapes)
+        want = [0] + ([5] if small else []) + ([8] if mid else [])
+        if large:
+            want += [1, 2, 3] * 9 + [1, 2, 4]
+        assert launch_list(lib, shapes, prec) == want
