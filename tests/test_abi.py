@@ -370,3 +370,28 @@ if given is not None:
         if large:
             want += [1, 2, 3] * 9 + [1, 2, 4]
         assert launch_list(lib, shapes, prec) == want
+
+
+@pytest.mark.parametrize("compiler,flags", [("gcc", ["-std=c99", "-x", "c"]),
+                                            ("g++", ["-std=c++17", "-x", "c++"])])
+def test_headers_compile_as_plain_c_and_cpp(tmp_path, compiler, flags):
+    """The ABI headers need no CUDA or torch types: a C program that calls
+    every entry point (through pointers, never run) compiles warning-free."""
+    import shutil
+    import subprocess
+
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not installed")
+    src = tmp_path / "use_abi.c"
+    calls = "\n".join(f"  (void)&{name};" for name in header_symbols())
+    src.write_text(
+        "#include <string.h>\n"
+        "#include \"muon_step.h\"\n#include \"muon_adamw.h\"\n#include \"muon_shard.h\"\n"
+        "int main(void) {\n" + calls + "\n"
+        "  muon_param_t p;\n  muon_adamw_hyper_t h;\n  muon_shard_update_t u;\n"
+        "  memset(&p, 0, sizeof p);\n  memset(&h, 0, sizeof h);\n  memset(&u, 0, sizeof u);\n"
+        "  return (int)(sizeof p + sizeof h + sizeof u == 0);\n}\n")
+    out = subprocess.run([compiler, *flags, "-Wall", "-Wextra", "-Werror", "-I",
+                          os.path.join(ROOT, "include"), "-c", str(src), "-o",
+                          str(tmp_path / "use_abi.o")], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
