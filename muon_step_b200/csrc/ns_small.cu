@@ -62,6 +62,10 @@ __device__ __forceinline__ void gemm128(uint32_t d, uint32_t a_base, uint32_t b_
   }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Write 32 values of row `i` (columns 32 ch .. 32 ch + 31) as bf16.
 __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const float (&v)[32]) {
 #pragma unroll
@@ -240,9 +244,15 @@ __global__ void __launch_bounds__(kThreads, 2) ns_small_kernel(const __grid_cons
         gemm128(tmem, sB, sX, true);
         ptx::umma_commit(bar_mma);
       }
+      const bool last = (k + 1 == a.steps);
+      if (last && md.W) {
+        // the caller's weight into L2 while the last product and its
+        // epilogue run: the update below then waits on L2, not DRAM
+        const int64_t lines = (md.n * md.m + 31) / 32;  // 128-byte lines of W
+        for (int64_t ln = tid; ln < lines; ln += kThreads) prefetch_l2(md.W + ln * 32);
+      }
       wait_mma();
       if (!ok) break;
-      const bool last = (k + 1 == a.steps);
 #pragma unroll
       for (int j = 0; j < kHalfCols / 32; ++j) {
         float v[32];
@@ -301,24 +311,37 @@ __global__ void __launch_bounds__(kThreads, 2) ns_small_kernel(const __grid_cons
       const bool tr = md.transposed != 0;
       const int rows = tr ? c : r;  // caller rows
       const int cols = tr ? r : c;  // caller columns
-      for (int crow = warp; crow < rows; crow += kThreads / 32) {
-        float* Wr = md.W ? md.W + static_cast<int64_t>(crow) * md.m : nullptr;
-        float* Or = md.O ? md.O + static_cast<int64_t>(crow) * md.m : nullptr;
-        float w[kS / 32], o[kS / 32];
+      // two caller rows per pass (crow, crow + 8), every load before the
+      // first store, so that their round trips overlap
+      constexpr int kRowStride = kThreads / 32;
+      for (int crow0 = warp; crow0 < rows; crow0 += 2 * kRowStride) {
+        float w[2][kS / 32], o[2][kS / 32];
 #pragma unroll
-        for (int q = 0; q < kS / 32; ++q) {
-          const int col = 32 * q + lane;
-          const int i = tr ? col : crow;  // iterate coordinates of caller (crow, col)
-          const int j = tr ? crow : col;
-          o[q] = T[i * kS + (j ^ (i & 31))];
-          w[q] = (col < cols && Wr) ? Wr[col] : 0.f;
+        for (int u = 0; u < 2; ++u) {
+          const int crow = crow0 + u * kRowStride;
+          const float* Wr = (md.W && crow < rows) ? md.W + static_cast<int64_t>(crow) * md.m : nullptr;
+#pragma unroll
+          for (int q = 0; q < kS / 32; ++q) {
+            const int col = 32 * q + lane;
+            const int i = tr ? col : crow;  // iterate coordinates of caller (crow, col)
+            const int j = tr ? crow : col;
+            o[u][q] = T[(i & (kS - 1)) * kS + ((j & (kS - 1)) ^ (i & 31))];
+            w[u][q] = (col < cols && Wr) ? Wr[col] : 0.f;
+          }
         }
 #pragma unroll
-        for (int q = 0; q < kS / 32; ++q) {
-          const int col = 32 * q + lane;
-          if (col >= cols) continue;
-          if (Or) Or[col] = o[q];
-          if (Wr) Wr[col] = fmaf(w[q], uc.keep, -uc.step * o[q]);
+        for (int u = 0; u < 2; ++u) {
+          const int crow = crow0 + u * kRowStride;
+          if (crow >= rows) break;
+          float* Wr = md.W ? md.W + static_cast<int64_t>(crow) * md.m : nullptr;
+          float* Or = md.O ? md.O + static_cast<int64_t>(crow) * md.m : nullptr;
+#pragma unroll
+          for (int q = 0; q < kS / 32; ++q) {
+            const int col = 32 * q + lane;
+            if (col >= cols) continue;
+            if (Or) Or[col] = o[u][q];
+            if (Wr) Wr[col] = fmaf(w[u][q], uc.keep, -uc.step * o[u][q]);
+          }
         }
       }
     }
