@@ -34,6 +34,13 @@
  *     per-device error word that muon_sync_status() reports and clears.
  *   - NaN / Inf in the inputs are not checked; they propagate as in the
  *     plain definition.
+ *   - Host threads: the library-wide setters (muon_set_wait_limit_ns,
+ *     muon_set_tracing) and the one-shot calls may be used from any thread.
+ *     A plan holds no lock: calls on one plan (execute, the set_* calls,
+ *     destroy) must not overlap in time. Work that runs concurrently must
+ *     not share a workspace. The device error word is shared by every caller
+ *     on a device, so muon_sync_status() reports and clears the errors of
+ *     all of them.
  */
 #ifndef MUON_STEP_H
 #define MUON_STEP_H

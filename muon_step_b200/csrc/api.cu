@@ -37,7 +37,7 @@ std::mutex g_mutex;
 int* g_err_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
-uint64_t g_wait_limit_ns = 2000000000ull;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};  // set from any host thread
 
 // Per-device setup: the error word's device address and the SM count.
 muon_status_t device_setup(int* dev_out) {
@@ -626,7 +626,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   const auto* mats = reinterpret_cast<const MatDesc*>(ws + plan->off_mats);
   float* scale = reinterpret_cast<float*>(ws + plan->off_scale);
   int* err = g_err_ptr[dev];
-  const uint64_t limit = g_wait_limit_ns;
+  const uint64_t limit = g_wait_limit_ns.load(std::memory_order_relaxed);
 
   EwArgs ew{};
   ew.groups = groups;
@@ -882,7 +882,9 @@ const char* muon_status_string(muon_status_t status) {
 
 int muon_abi_version(void) { return MUON_ABI_VERSION; }
 
-void muon_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns < 1000 ? 1000 : ns; }
+void muon_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns < 1000 ? 1000 : ns, std::memory_order_relaxed);
+}
 
 muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream) {
   if (!flag) return MUON_ERR_INVALID_ARG;
