@@ -64,6 +64,26 @@ def _matrix(t: torch.Tensor, name: str) -> torch.Tensor:
     return t
 
 
+def _one_device(tensors, what="matrices"):
+    """The common device of the tensors (None entries skipped); raise if they differ."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all {what} must be on one CUDA device, got {sorted(map(str, devs))}")
+    return devs.pop()
+
+
+def _workspace(ws, device):
+    """(pointer, size in bytes) of a caller's workspace: a contiguous CUDA
+    tensor of any dtype on `device`."""
+    if not isinstance(ws, torch.Tensor) or ws.device.type != "cuda":
+        raise TypeError("workspace must be a CUDA tensor")
+    if not ws.is_contiguous():
+        raise TypeError("workspace must be contiguous")
+    if ws.device != device:
+        raise ValueError(f"workspace is on {ws.device}, the matrices on {device}")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
 def _schedule(schedule, eps):
     """(struct or None, keep-alive array)."""
     if schedule is None and eps is None:
@@ -144,8 +164,6 @@ class _PlanBase:
             if getattr(self, "_own_ws", None) is None:
                 self._own_ws = self.alloc_workspace()
             workspace = self._own_ws
-        if workspace.device.type != "cuda":
-            raise TypeError("workspace must be a CUDA tensor")
         return workspace
 
 
@@ -169,7 +187,7 @@ class MuonPlan(_PlanBase):
             self._tensors.append((W, G, M, O))
         if not items:
             raise ValueError("no matrices")
-        self.device = self._tensors[0][0].device
+        self.device = _one_device([t for q in self._tensors for t in q])
         arr = (MuonParam * len(items))(*items)
         sched, self._sched_keep = _schedule(schedule, eps)
         plan = ctypes.c_void_p()
@@ -216,10 +234,10 @@ class MuonPlan(_PlanBase):
 
     def execute(self, workspace=None, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2,
                 nesterov=True, stream=None):
-        workspace = self._ws(workspace)
+        ptr, nbytes = _workspace(self._ws(workspace), self.device)
         h = MuonHyper(lr, momentum, weight_decay, gamma, 1 if nesterov else 0)
-        _check(_lib.load().muon_plan_execute(self._plan, ctypes.byref(h), workspace.data_ptr(),
-                                             workspace.numel(), _stream_ptr(stream)),
+        _check(_lib.load().muon_plan_execute(self._plan, ctypes.byref(h), ptr, nbytes,
+                                             _stream_ptr(stream)),
                "muon_plan_execute")
 
 
@@ -238,7 +256,7 @@ class NsPlan(_PlanBase):
             self._tensors.append((X, O))
         if not items:
             raise ValueError("no matrices")
-        self.device = self._tensors[0][0].device
+        self.device = _one_device([t for q in self._tensors for t in q])
         arr = (MuonNsMatrix * len(items))(*items)
         sched, self._sched_keep = _schedule(schedule, eps)
         plan = ctypes.c_void_p()
@@ -249,9 +267,8 @@ class NsPlan(_PlanBase):
         self._destroy = _lib.load().muon_plan_destroy
 
     def execute(self, workspace=None, stream=None):
-        workspace = self._ws(workspace)
-        _check(_lib.load().muon_plan_execute(self._plan, None, workspace.data_ptr(),
-                                             workspace.numel(), _stream_ptr(stream)),
+        ptr, nbytes = _workspace(self._ws(workspace), self.device)
+        _check(_lib.load().muon_plan_execute(self._plan, None, ptr, nbytes, _stream_ptr(stream)),
                "muon_plan_execute")
 
 
@@ -263,22 +280,28 @@ def muon_step(params, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, neste
     for k, p in enumerate(params):
         W, G, M = (_matrix(t, f"params[{k}].{nm}") for t, nm in zip(p[:3], "WGM"))
         O = p[3] if len(p) > 3 else None
-        if not (W.shape == G.shape == M.shape):
-            raise ValueError(f"params[{k}]: W, G, M must have one shape")
-        keep.append(p)
+        if O is not None:
+            _matrix(O, f"params[{k}].O")
+        if not (W.shape == G.shape == M.shape and (O is None or O.shape == W.shape)):
+            raise ValueError(f"params[{k}]: W, G, M (and O) must have one shape")
+        keep.append((W, G, M, O))
         items.append(MuonParam(W.data_ptr(), G.data_ptr(), M.data_ptr(),
                                O.data_ptr() if O is not None else None, *W.shape))
+    if not items:
+        raise ValueError("no matrices")
+    device = _one_device([t for q in keep for t in q])
     arr = (MuonParam * len(items))(*items)
     lib = _lib.load()
     prec = _precision(precision)
     if workspace is None:
         n = ctypes.c_size_t()
         _check(lib.muon_workspace_size(arr, len(items), prec, ctypes.byref(n)), "muon_workspace_size")
-        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=keep[0][0].device)
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=device)
+    ptr, nbytes = _workspace(workspace, device)
     sched, _keep = _schedule(schedule, eps)
     _check(lib.muon_step(arr, len(items), lr, momentum, weight_decay, gamma, 1 if nesterov else 0,
-                         ctypes.byref(sched) if sched else None, prec, workspace.data_ptr(),
-                         workspace.numel(), _stream_ptr(stream)), "muon_step")
+                         ctypes.byref(sched) if sched else None, prec, ptr, nbytes,
+                         _stream_ptr(stream)), "muon_step")
     return workspace
 
 
@@ -286,7 +309,15 @@ def ns_orthogonalize(xs, out=None, precision="bf16", schedule=None, eps=None, wo
                      stream=None):
     """O' = NewtonSchulz(X / (||X||_F + eps)) per matrix (C ABI ns_orthogonalize)."""
     xs = [_matrix(x, f"X[{k}]") for k, x in enumerate(xs)]
-    out = [torch.empty_like(x) for x in xs] if out is None else list(out)
+    if not xs:
+        raise ValueError("no matrices")
+    if out is None:
+        out = [torch.empty_like(x) for x in xs]
+    else:
+        out = [_matrix(o, f"out[{k}]") for k, o in enumerate(out)]
+        if len(out) != len(xs) or any(o.shape != x.shape for x, o in zip(xs, out)):
+            raise ValueError("out must hold one matrix of X's shape per input")
+    device = _one_device(xs + out)
     items = (MuonNsMatrix * len(xs))(*[MuonNsMatrix(x.data_ptr(), o.data_ptr(), *x.shape)
                                        for x, o in zip(xs, out)])
     lib = _lib.load()
@@ -294,10 +325,11 @@ def ns_orthogonalize(xs, out=None, precision="bf16", schedule=None, eps=None, wo
     if workspace is None:
         n = ctypes.c_size_t()
         _check(lib.ns_workspace_size(items, len(xs), prec, ctypes.byref(n)), "ns_workspace_size")
-        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=xs[0].device)
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=device)
+    ptr, nbytes = _workspace(workspace, device)
     sched, _keep = _schedule(schedule, eps)
     _check(lib.ns_orthogonalize(items, len(xs), ctypes.byref(sched) if sched else None, prec,
-                                workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
+                                ptr, nbytes, _stream_ptr(stream)),
            "ns_orthogonalize")
     return out
 
@@ -320,6 +352,7 @@ def _adamw_items(params):
         keep.append((p, g, m, v))
     if not items:
         raise ValueError("no tensors")
+    _one_device([t for q in keep for t in q], "tensors")
     return (AdamwParam * len(items))(*items), keep
 
 
@@ -382,9 +415,12 @@ class AdamWPlan:
             if self._ws_cache is None:
                 self._ws_cache = self.alloc_workspace()
             workspace = self._ws_cache
+        ptr, nbytes = _workspace(workspace, self.device)
+        if step_tensor is not None and step_tensor.device != self.device:
+            raise ValueError(f"step_tensor is on {step_tensor.device}, the tensors on {self.device}")
         h = _adamw_hyper(lr, betas, eps, weight_decay, step, step_tensor)
-        _check(_lib.load().muon_adamw_plan_execute(self._plan, ctypes.byref(h), workspace.data_ptr(),
-                                                   workspace.numel(), _stream_ptr(stream)),
+        _check(_lib.load().muon_adamw_plan_execute(self._plan, ctypes.byref(h), ptr, nbytes,
+                                                   _stream_ptr(stream)),
                "muon_adamw_plan_execute")
 
 
@@ -398,9 +434,10 @@ def adamw_step(params, step, lr=0.02, betas=(0.9, 0.999), eps=1e-8, weight_decay
         _check(lib.muon_adamw_workspace_size(arr, len(arr), ctypes.byref(n)),
                "muon_adamw_workspace_size")
         workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=keep[0][0].device)
+    ptr, nbytes = _workspace(workspace, keep[0][0].device)
     h = _adamw_hyper(lr, betas, eps, weight_decay, step, None)
-    _check(lib.muon_adamw_step(arr, len(arr), ctypes.byref(h), workspace.data_ptr(),
-                               workspace.numel(), _stream_ptr(stream)), "muon_adamw_step")
+    _check(lib.muon_adamw_step(arr, len(arr), ctypes.byref(h), ptr, nbytes, _stream_ptr(stream)),
+           "muon_adamw_step")
     return workspace
 
 
