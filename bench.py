@@ -29,6 +29,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -127,19 +128,112 @@ def cpu_oracle_rate(wl_cpu_mats, hyper, budget_s=None):
     return metric_flops(done) / dt / 1e12, dt, len(done)
 
 
+def _nvml_uuid(local_rank):
+    """NVML's name for the CUDA device, "GPU-<uuid>", or None."""
+    try:
+        import torch
+        return "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        return None
+
+
+class NvmlClockReader:
+    """SM clock and clock-event reasons of one GPU, read through NVML every
+    `period_s` seconds in a background thread, with host timestamps. Read-only
+    queries; any NVML failure leaves the reader without samples."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, index, uuid=None, period_s=0.01, nvml=None):
+        self.index, self.uuid, self.period_s = index, uuid, period_s
+        self.nvml = nvml
+        self.samples = []  # (monotonic time, SM MHz, reason bit mask)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def start(self):
+        try:
+            if self.nvml is None:
+                import pynvml
+                self.nvml = pynvml
+            nv = self.nvml
+            nv.nvmlInit()
+            handle = None
+            if self.uuid:
+                try:
+                    handle = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+                except Exception:
+                    handle = None
+            if handle is None:
+                handle = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM))
+            reasons = (getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                       or nv.nvmlDeviceGetCurrentClocksThrottleReasons)
+        except Exception:
+            self.nvml = None
+            return False
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((time.monotonic(),
+                                         float(nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)),
+                                         int(reasons(handle))))
+                except Exception:
+                    return
+                self._stop.wait(self.period_s)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+        return True
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2.0)
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+
+    def summary(self, t0, t1):
+        """Median SM clock and the reasons seen between host times t0 and t1
+        (None without samples there)."""
+        win = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+        if not win:
+            return None
+        reasons = sorted({nm for _, _, mask in win for nm, bit in self.REASONS if mask & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win), "source": "nvml, timed region"}
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms from before
+    the warm-up to the end of the timed region, and NVML read every 10 ms
+    inside the timed region (used when it has samples there)."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, uuid=None, nvml=None):
         self.index = index
         self.proc = None
         self.path = None
+        self.reader = NvmlClockReader(index, uuid=uuid, nvml=nvml)
+        self.t0 = self.t1 = None
+
+    def window_begin(self):
+        self.t0 = time.monotonic()
+
+    def window_end(self):
+        self.t1 = time.monotonic()
 
     def start(self):
+        self.reader.start()
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -152,6 +246,15 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        self.reader.stop()
+        smi = self._stop_smi()
+        nv = self.reader.summary(self.t0, self.t1)
+        if nv is None:
+            return smi
+        nv["smi_samples"] = smi.get("samples", 0)
+        return nv
+
+    def _stop_smi(self):
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         self.proc.terminate()
@@ -177,7 +280,8 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvidia-smi, warm-up and timed region"}
 
 
 KERNEL_SOURCES = ("muon_step_b200/csrc/ns_tc.cu", "muon_step_b200/csrc/ptx_sm100.cuh",
@@ -345,7 +449,7 @@ def main():
         plan.execute(ws, lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"], gamma=h["gamma"],
                      nesterov=h["nesterov"], stream=stream)
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(local_rank, uuid=_nvml_uuid(local_rank))
     clocks.start()
     for _ in range(max(args.warmup, 0)):
         step()
@@ -380,6 +484,7 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    clocks.window_begin()
     t_start.record(stream)
     if graph is not None:
         graph.replay()
@@ -389,6 +494,7 @@ def main():
             step()
     t_end.record(stream)
     torch.cuda.synchronize()
+    clocks.window_end()
     barrier()
     plan.set_events(None)
     clk = clocks.stop()
