@@ -8,9 +8,9 @@ the learning rate and the weight decay.
 
 Both groups run in the library's kernels: one Muon plan (MuonPlan) and one
 AdamW plan (AdamWPlan), executed on the same stream. Plans record pointers, so
-gradients must stay in place between steps (accumulate into .grad, zero it
-with ``zero_grad(set_to_none=False)``); if a gradient tensor is replaced, the
-next step rebuilds the plans.
+gradients should stay in place between steps (accumulate into .grad, zero it
+with ``zero_grad()`` here); if a parameter's or a gradient's storage is
+replaced, the next step rebuilds the plans.
 """
 
 from __future__ import annotations
@@ -44,6 +44,35 @@ def route(named_shapes: Iterable[Tuple[str, Sequence[int]]],
     return muon, adamw
 
 
+def route_module(model, adamw_names: Sequence[str] = ()):
+    """Split a module's parameters between Muon and AdamW by what they are.
+
+    AdamW: the weights of embedding tables (torch.nn.Embedding); a linear
+    layer's weight that is the same tensor as an embedding's (a tied
+    prediction head) or whose output width is an embedding's vocabulary size
+    (an untied head); every parameter that is not 2-D; and names containing
+    any of ``adamw_names`` (case-insensitive). Muon: every other 2-D
+    parameter. Names follow ``model.named_parameters()`` (a tied tensor is
+    listed once, under its first name). Returns (muon_names, adamw_names).
+    """
+    import torch.nn as nn
+
+    tables = [m for m in model.modules() if isinstance(m, nn.Embedding)]
+    table_ids = {id(m.weight) for m in tables}
+    vocab = {m.num_embeddings for m in tables}
+    head_ids = set()
+    for m in model.modules():
+        if isinstance(m, nn.Linear) and (id(m.weight) in table_ids or m.out_features in vocab):
+            head_ids.add(id(m.weight))
+    tags = tuple(t.lower() for t in adamw_names)
+    muon, adamw = [], []
+    for name, p in model.named_parameters():
+        to_adamw = (p.dim() != 2 or id(p) in table_ids or id(p) in head_ids
+                    or any(t in name.lower() for t in tags))
+        (adamw if to_adamw else muon).append(name)
+    return muon, adamw
+
+
 class HybridOptimizer:
     """Muon + AdamW over a model's named parameters (float32 CUDA tensors).
 
@@ -54,12 +83,24 @@ class HybridOptimizer:
     def __init__(self, named_params: Iterable[Tuple[str, torch.Tensor]], lr=0.02, momentum=0.95,
                  weight_decay=0.1, gamma=0.2, nesterov=True, betas=(0.9, 0.999), eps=1e-8,
                  precision="bf16", schedule=None, scale_mode="shape",
-                 adamw_names: Sequence[str] = DEFAULT_ADAMW_NAMES):
+                 adamw_names: Sequence[str] = DEFAULT_ADAMW_NAMES,
+                 muon_names: Optional[Sequence[str]] = None):
         params = list(named_params)
         if not params:
             raise ValueError("no parameters")
         by_name = dict(params)
-        muon_names, adamw_names_ = route(((n, p.shape) for n, p in params), adamw_names)
+        if muon_names is None:
+            muon_names, adamw_names_ = route(((n, p.shape) for n, p in params), adamw_names)
+        else:
+            chosen = set(muon_names)
+            unknown = chosen - set(by_name)
+            if unknown:
+                raise ValueError(f"unknown parameter names: {sorted(unknown)}")
+            bad = [n for n in chosen if by_name[n].dim() != 2]
+            if bad:
+                raise ValueError(f"Muon parameters must be 2-D: {sorted(bad)}")
+            muon_names = [n for n, _ in params if n in chosen]
+            adamw_names_ = [n for n, _ in params if n not in chosen]
         self.muon_params = [(n, by_name[n]) for n in muon_names]
         self.adamw_params = [(n, by_name[n]) for n in adamw_names_]
         self.hyper = dict(lr=lr, momentum=momentum, weight_decay=weight_decay, gamma=gamma,
@@ -69,18 +110,26 @@ class HybridOptimizer:
         self.exp_avg = {n: torch.zeros_like(p) for n, p in self.adamw_params}
         self.exp_avg_sq = {n: torch.zeros_like(p) for n, p in self.adamw_params}
         self.step_count = 0
-        self._grad_ptrs = None
+        self._ptrs = None
         self._muon = self._adamw = None
         self._muon_ws = self._adamw_ws = None
         self._diag: Optional[torch.Tensor] = None
 
+    @classmethod
+    def from_module(cls, model, adamw_names: Sequence[str] = (), **kw):
+        """A HybridOptimizer over ``model``'s parameters, split by
+        ``route_module`` (embedding tables and prediction heads on AdamW)."""
+        muon, _ = route_module(model, adamw_names)
+        return cls(model.named_parameters(), muon_names=muon, **kw)
+
     # ------------------------------------------------------------------ plans
-    def _current_grad_ptrs(self):
+    def _current_ptrs(self):
+        """The parameter and gradient addresses the plans were built on."""
         ptrs = []
         for n, p in self.muon_params + self.adamw_params:
             if p.grad is None:
                 raise RuntimeError(f"parameter {n!r} has no gradient")
-            ptrs.append(p.grad.data_ptr())
+            ptrs.append((p.data_ptr(), p.grad.data_ptr()))
         return tuple(ptrs)
 
     def _build(self):
@@ -115,10 +164,10 @@ class HybridOptimizer:
     # ------------------------------------------------------------------ step
     def step(self, stream=None):
         """One step of both groups on `stream` (default: the current stream)."""
-        ptrs = self._current_grad_ptrs()
-        if ptrs != self._grad_ptrs:
+        ptrs = self._current_ptrs()
+        if ptrs != self._ptrs:
             self._build()
-            self._grad_ptrs = ptrs
+            self._ptrs = ptrs
         self.step_count += 1
         h = self.hyper
         if self._muon is not None:

@@ -286,3 +286,71 @@ def test_many_small_tensors_in_bundles():
     for k, (p, m, v) in enumerate(state):
         for got, want in ((p, ref[k][0]), (m, ref[k][1]), (v, ref[k][2])):
             assert _rel(got.double().cpu().numpy(), want) <= TOL, sizes[k]
+
+
+def _gpt2_like(tied=True):
+    import torch.nn as nn
+
+    class Block(nn.Module):
+        def __init__(self):
+            super().__init__()
+            self.ln = nn.LayerNorm(16)
+            self.multi_head_attn = nn.Linear(16, 48)
+            self.mlp = nn.Linear(16, 64)
+
+    class Model(nn.Module):
+        def __init__(self):
+            super().__init__()
+            self.wte = nn.Embedding(100, 16)
+            self.wpe = nn.Embedding(32, 16)
+            self.h = nn.ModuleList([Block()])
+            self.out = nn.Linear(16, 100, bias=False)
+            if tied:
+                self.out.weight = self.wte.weight
+
+    return Model()
+
+
+def test_route_module_puts_tables_and_heads_on_adamw():
+    from muon_step_b200.hybrid import route_module
+
+    muon, adamw = route_module(_gpt2_like(tied=True))
+    assert muon == ["h.0.multi_head_attn.weight", "h.0.mlp.weight"]
+    assert adamw == ["wte.weight", "wpe.weight", "h.0.ln.weight", "h.0.ln.bias",
+                     "h.0.multi_head_attn.bias", "h.0.mlp.bias"]
+    muon, adamw = route_module(_gpt2_like(tied=False))
+    assert muon == ["h.0.multi_head_attn.weight", "h.0.mlp.weight"]
+    assert "out.weight" in adamw                      # untied head: output width = vocabulary
+    muon, _ = route_module(_gpt2_like(tied=False), adamw_names=("mlp",))
+    assert muon == ["h.0.multi_head_attn.weight"]
+
+
+def test_hybrid_from_module_and_explicit_split():
+    from muon_step_b200.hybrid import HybridOptimizer
+
+    model = _gpt2_like()
+    opt = HybridOptimizer.from_module(model)
+    assert [n for n, _ in opt.muon_params] == ["h.0.multi_head_attn.weight", "h.0.mlp.weight"]
+    assert len(opt.adamw_params) == 6
+    with pytest.raises(ValueError):
+        HybridOptimizer(model.named_parameters(), muon_names=["nope.weight"])
+    with pytest.raises(ValueError):
+        HybridOptimizer(model.named_parameters(), muon_names=["h.0.mlp.bias"])
+
+
+def test_hybrid_rebuilds_when_a_parameter_moves():
+    import torch
+
+    from muon_step_b200.hybrid import HybridOptimizer
+
+    w = torch.nn.Parameter(torch.zeros(8, 8))
+    b = torch.nn.Parameter(torch.zeros(8))
+    w.grad, b.grad = torch.zeros(8, 8), torch.zeros(8)
+    opt = HybridOptimizer([("w", w), ("b", b)])
+    key = opt._current_ptrs()
+    assert opt._current_ptrs() == key
+    w.data = torch.ones(8, 8)            # new storage for the parameter
+    assert opt._current_ptrs() != key
+    key = opt._current_ptrs()
+    b.grad = torch.ones(8)               # new storage for a gradient
+    assert opt._current_ptrs() != key
