@@ -82,7 +82,7 @@ typedef struct {
   const float* G; /* n x m gradient, read only */
   float* M;       /* n x m momentum buffer, updated in place */
   float* O;       /* optional n x m output of O' (before the RMS rescale); NULL to skip */
-  int64_t n, m;   /* 1 <= n, m <= 2^31 - 1 */
+  int64_t n, m;   /* 1 <= n, m <= 2^31 - 8 */
 } muon_param_t;
 
 /* Newton-Schulz schedule ([V4-book] §4). `abc` is a HOST array of steps * 3
@@ -99,7 +99,7 @@ typedef struct {
 typedef struct {
   const float* X; /* n x m input, read only */
   float* O;       /* n x m output, must not overlap X */
-  int64_t n, m;
+  int64_t n, m;   /* 1 <= n, m <= 2^31 - 8 */
 } muon_ns_matrix_t;
 
 /* Hyper-parameters of one step ([V4-breakdown] Algorithm 1: eta, mu, lambda,

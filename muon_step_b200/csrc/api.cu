@@ -408,8 +408,12 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   return MUON_OK;
 }
 
+// The planner keeps r, c and their leading dimensions (rounded up to 8) in
+// 32-bit fields, so both sides stop 8 short of 2^31.
+constexpr int64_t kMaxDim = 0x7fffffffLL - 7;
+
 bool valid_shape(int64_t n, int64_t m) {
-  return n >= 1 && m >= 1 && n <= 0x7fffffffLL && m <= 0x7fffffffLL;
+  return n >= 1 && m >= 1 && n <= kMaxDim && m <= kMaxDim;
 }
 
 muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {

@@ -78,6 +78,9 @@ def test_plan_rejects_bad_arguments(lib):
     assert lib.muon_plan_create(params([(4, 4)]), 1, 7, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
     assert lib.muon_plan_create(params([(0, 4)]), 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
     assert lib.muon_plan_create(params([(4, -1)]), 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
+    # a side above 2^31 - 8 would overflow the 32-bit leading dimension
+    for shape in [(1, 2 ** 31 - 7), (2 ** 31 - 1, 1), (1, 2 ** 40)]:
+        assert lib.muon_plan_create(params([shape]), 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
     bad = params([(4, 4)])
     bad[0].G = None
     assert lib.muon_plan_create(bad, 1, 0, None, ctypes.byref(plan)) == MUON_ERR_INVALID_ARG
