@@ -14,10 +14,10 @@
 // significant bits; in fp32 mode as fp32.
 //
 // HBM-bound: each element reads G and M (8 B) and writes M and the two bf16
-// parts (8 B; fp32 mode: M and the fp32 iterate). Tiles are 64 x 128 elements; a tile's threads
-// read and write whole 128-byte lines (64 x 128 elements). When the iterate is the transpose, the
-// tile is staged in shared memory so that the transposed writes stay
-// coalesced. Per-tile partial sums of squares go to a buffer; the last tile of
+// parts (8 B; fp32 mode: M and the fp32 iterate). Tiles are 64 x 128
+// elements, and a tile's threads read and write whole 128-byte lines. When
+// the iterate is the transpose, the tile is staged in shared memory so that
+// the transposed writes stay coalesced. Per-tile partial sums of squares go to a buffer; the last tile of
 // each matrix to finish (arrival counter) adds them in a fixed order, in
 // double, so the norm is deterministic.
 //
