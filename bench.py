@@ -4,15 +4,19 @@
 A step is the whole hot path over one batch of matrices: momentum + Nesterov +
 Frobenius norm + cast (1 kernel), then 10 hybrid Newton-Schulz steps (3 grouped
 GEMM kernels each), the last one fused with the RMS rescale, decoupled weight
-decay and parameter update. Default workload: 64 square 1024 x 1024 fp32
-matrices (W, G, M resident in HBM, 805 MB, larger than the 126 MB L2, so no
-explicit L2 flush between steps), bf16 Newton-Schulz operands.
+decay and parameter update. Default workload: the dense transformer stack of
+16 layers at d = 4096 (per layer Q, K, V, O 4096 x 4096, gate and up 4096 x
+14336, down 14336 x 4096 on the transposed path: 112 fp32 matrices, W, G and M
+resident in HBM, 46.7 GB, far larger than the 126 MB L2, so no explicit L2
+flush between steps), bf16 Newton-Schulz operands. `--config batch64_1024`
+runs 64 square 1024 x 1024 matrices instead.
 
 Metric: Newton-Schulz TFLOP/s of the whole step, with the FLOPs the metric
 defines, 10 (4 r^2 c + 2 r^3) per matrix (r = min(n, m), c = max(n, m)), and
-the step time in ms. Multi-GPU: every rank runs its own batch (independent
-problems, no data-path collective, weak scaling); value = FLOPs of all ranks /
-the slowest rank's time.
+the step time in ms. The roofline of the dominant kernel counts the FLOPs its
+tiles execute (the symmetric stages skip the upper tiles). Multi-GPU: every
+rank runs its own batch (independent problems, no data-path collective, weak
+scaling); value = FLOPs of all ranks / the slowest rank's time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
     python bench.py --impl reference     # the float64 CPU oracle, timed on a sample
@@ -48,7 +52,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="batch64_1024")
+    ap.add_argument("--config", default="dense_d4096")
     ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
@@ -75,6 +79,107 @@ def apply_bytes(shapes):
     iterate (bf16 high + low parts, r x c) read once and written once:
     2 r^2 + 8 r c per matrix."""
     return sum(2.0 * min(n, m) ** 2 + 8.0 * min(n, m) * max(n, m) for n, m in shapes)
+
+
+TINY_ELEMS = 4096  # matrices of at most this many elements: the tiny fp32 kernel
+
+
+def one_cta_kind(n, m, precision="bf16"):
+    """Launch kind of the one-CTA kernel that runs a matrix (5 small, 8 mid,
+    9 tiny), or None when it takes the grouped stage kernels."""
+    if precision != "bf16":
+        return None
+    r, c = min(n, m), max(n, m)
+    if r * c <= TINY_ELEMS:
+        return 9
+    if r <= 128 and c <= 128:
+        return 5
+    if r <= 128 and c <= 512:
+        return 8
+    return None
+
+
+def stage_bytes(kind, shapes, precision="bf16"):
+    """Algorithmic HBM bytes of one launch of a grouped stage over these
+    matrices: each operand read once, each result written once.
+                   bf16 operands                               fp32 operands
+      Gram (1)     X high part read, A written: 2rc + 2r^2     X read, A written: 4rc + 4r^2
+      Poly (2)     A read, B written: 4r^2                     8r^2
+      Apply (3)    B read, X high + low in and out: 2r^2 + 8rc B read, X in and out: 4r^2 + 8rc
+      ApplyLast(4) B, X in, W read and written: 2r^2 + 12rc    4r^2 + 12rc"""
+    f = 2.0 if precision == "bf16" else 4.0
+    tot = 0.0
+    for n, m in shapes:
+        r, c = float(min(n, m)), float(max(n, m))
+        tot += {1: f * r * c + f * r * r, 2: 2 * f * r * r, 3: f * r * r + 8 * r * c,
+                4: f * r * r + 12 * r * c}[kind]
+    return tot
+
+
+def executed_stage_flops(kind, shapes, precision="bf16"):
+    """FLOPs one launch of a grouped stage executes over these matrices. With
+    bf16 operands the symmetric stages (Gram, Poly) run only the 128 x 128
+    blocks on or below the diagonal, clipped to the matrix; the fp32 kernels
+    and Apply run the whole product."""
+    tot = 0.0
+    for n, m in shapes:
+        r, c = min(n, m), max(n, m)
+        if kind in (3, 4) or precision != "bf16":
+            tot += 2.0 * r * r * (r if kind == 2 else c)
+            continue
+        k = c if kind == 1 else r
+        rb = -(-r // 128)
+        for i in range(rb):
+            rows = min(128, r - 128 * i)
+            for j in range(i + 1):
+                tot += 2.0 * rows * min(128, r - 128 * j) * k
+    return tot
+
+
+def dominant_roofline(kinds, per_kind_ms, shapes, peaks, precision="bf16", ns_steps=10):
+    """Roofline record of the kernel kind with the largest total time.
+
+    per_kind_ms maps a launch kind to the list of its launch durations (ms).
+    Bytes and FLOPs are per launch and algorithmic: the grouped stages by
+    stage_bytes / executed_stage_flops over the matrices they run; the
+    elementwise kernel 16 B per element of every matrix; a one-CTA kernel
+    12 B per element (iterate high and low parts in, W in and out) and every
+    step's FLOPs. The bound is whichever of FLOPs at the sustained bf16 peak
+    or bytes at the HBM copy bandwidth takes longer."""
+    share = {k: sum(v) for k, v in per_kind_ms.items()}
+    dom = max(share, key=lambda k: share[k])
+    avg_ms = share[dom] / len(per_kind_ms[dom])
+    stage = "stage_tc_kernel" if precision == "bf16" else "stage_simt_kernel"
+    names = {0: "ew_kernel", 1: f"{stage}<Gram>", 2: f"{stage}<Poly>", 3: f"{stage}<Apply>",
+             4: f"{stage}<ApplyLast>", 5: "ns_small_kernel", 8: "ns_mid_kernel",
+             9: "ns_tiny_kernel", 6: "rms_reduce_kernel", 7: "finish_kernel"}
+    grouped = [(n, m) for n, m in shapes if one_cta_kind(n, m, precision) is None]
+    if dom in (1, 2, 3, 4):
+        flops = executed_stage_flops(dom, grouped, precision)
+        nbytes = stage_bytes(dom, grouped, precision)
+    elif dom in (5, 8, 9):
+        mine = [(n, m) for n, m in shapes if one_cta_kind(n, m, precision) == dom]
+        flops = sum(ns_steps * (4.0 * min(n, m) ** 2 * max(n, m) + 2.0 * min(n, m) ** 3)
+                    for n, m in mine)
+        nbytes = sum(12.0 * n * m for n, m in mine)
+    else:
+        flops = 0.0
+        nbytes = sum(16.0 * n * m for n, m in shapes)
+    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    hbm_peak = float(peaks["hbm_gbs"])
+    t_tensor = flops / (tensor_peak * 1e12)
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    if t_hbm >= t_tensor:
+        achieved = nbytes / (avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak}
+    else:
+        achieved = flops / (avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak}
+    roof.update({"kind": dom, "kernel": names.get(dom, str(dom)), "launch_ms": avg_ms,
+                 "flops_per_launch": flops, "bytes_per_launch": nbytes})
+    return roof
 
 
 def max_over_ranks(x, device, world):
@@ -297,14 +402,18 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(config):
-    """Per-launch DRAM bytes of the Apply kernel from the committed ncu summary,
-    or None when there is none for this workload or the kernel sources changed
-    since the counters were taken."""
+def traffic_from_profile(config, kind=3):
+    """Per-launch DRAM bytes of the dominant stage kernel (launch kind `kind`)
+    from the committed ncu summary of this workload, or None when there is
+    none, it covers another kernel, or the kernel sources changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", f"ns_stages_{config}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
+    k = re.search(r"^traffic_kind:\s*([0-9]+)\s*$", text, re.M)
+    if (int(k.group(1)) if k else 3) != kind:
+        return None
     m = re.search(r"^traffic_per_launch_bytes:\s*([0-9.eE+]+)\s*$", text, re.M)
     h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)\s*$", text, re.M)
     if not m or not h or h.group(1) != kernel_source_hash():
@@ -520,39 +629,11 @@ def main():
     peaks, peak_src = load_peaks()
     g_fl, p_fl, a_fl = plan.flops()
     tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    hbm_peak = float(peaks["hbm_gbs"])
-    if 3 in avg:
-        # the dominant kernel: the grouped Apply stage
-        dom_flops = a_fl / ns_steps
-        dom_bytes = apply_bytes(wl.shapes)
-        dom_ms = avg[3]
-        dom_name = "stage_tc_kernel<Apply>" if args.precision == "bf16" else "stage_simt_kernel<Apply>"
-        traffic = traffic_from_profile(args.config)
-    else:
-        # every matrix runs in the one-CTA kernels (all steps in one launch):
-        # the small-matrix (5) or the mid-size (8) kernel, whichever took longer;
-        # bytes: iterate high + low parts read, W read and written (12 B per element)
-        kd = max((k for k in (5, 8) if k in share), key=lambda k: share[k])
-        mine = [(n, m) for n, m in wl.shapes
-                if (max(n, m) <= 128) == (kd == 5) and min(n, m) <= 128 and max(n, m) <= 512]
-        dom_flops = sum(ns_steps * (4.0 * min(n, m) ** 2 * max(n, m) + 2.0 * min(n, m) ** 3)
-                        for n, m in mine)
-        dom_bytes = sum(12.0 * n * m for n, m in mine)
-        dom_ms = avg[kd]
-        dom_name = "ns_small_kernel" if kd == 5 else "ns_mid_kernel"
-        traffic = None
-    t_tensor = dom_flops / (tensor_peak * 1e12)
-    t_hbm = dom_bytes / (hbm_peak * 1e9)
-    if t_hbm >= t_tensor:
-        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": traffic}
-    else:
-        achieved = dom_flops / (dom_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak, "traffic": traffic}
-    roof["kernel"] = dom_name
+    burst_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roof = dominant_roofline(kinds, per_kind, wl.shapes, peaks, args.precision, ns_steps)
+    roof["traffic"] = traffic_from_profile(args.config, roof["kind"])
     roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'HBM copy'})"
+    executed = (g_fl + p_fl + a_fl) / (ms_per_step / 1e3) / 1e12
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -639,7 +720,7 @@ def main():
 
     if rank == 0:
         names = {0: "elementwise", 1: "gram", 2: "poly", 3: "apply", 4: "apply_update", 5: "small",
-                 6: "rms_reduce", 7: "update", 8: "mid"}
+                 6: "rms_reduce", 7: "update", 8: "mid", 9: "tiny"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -651,12 +732,13 @@ def main():
                        "l2": "inputs larger than L2 (no flush)" if wl.elements() * 12 > 126e6
                              else "inputs smaller than L2",
                        "metric_flops_per_step": flops_rank},
-            "pct_of_peak": {"bf16_burst": value / float(peaks.get("bf16_tflops", 1590.0)),
-                            "bf16_sustained": value / tensor_peak},
+            "pct_of_peak": {"dense_eq_of_burst": value / burst_peak,
+                            "executed_of_burst": executed / burst_peak,
+                            "executed_of_sustained": executed / tensor_peak},
             "roofline": roof,
             "kernels_ms_avg": {names[k]: v for k, v in sorted(avg.items())},
             "kernels_share": {names[k]: v / tot_kernel for k, v in sorted(share.items())},
-            "executed_tflops": (g_fl + p_fl + a_fl) / (ms_per_step / 1e3) / 1e12,
+            "executed_tflops": executed,
             "gpu_launches": len(kinds) * args.steps,
             "cuda_graph": graph is not None,
             "clocks": clk,

@@ -172,7 +172,10 @@ MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes)
 
 /* Run the plan: one kernel for momentum / norm / cast, then three kernels per
  * Newton-Schulz step, each one persistent launch over every matrix. `hyper` is
- * ignored (may be NULL) for an ns_orthogonalize plan. */
+ * ignored (may be NULL) for an ns_orthogonalize plan. The first execute on a
+ * workspace (or on another device) copies the plan's descriptor tables into
+ * it with cudaMemcpyAsync from host memory the plan owns: the plan must
+ * outlive that copy, and anything that repeats it. */
 MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
@@ -181,7 +184,9 @@ MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* h
  * 5 small-matrix kernel (all steps and the update of matrices up to
  * 128 x 128), 6 per-matrix RMS reduction, 7 update pass, 8 mid-size kernel
  * (all steps and the update of matrices with min(n, m) <= 128 < max(n, m)
- * <= 512)). */
+ * <= 512), 9 tiny-matrix kernel (bf16 precision only: matrices of at most
+ * 4096 elements run every step with fp32 operands, since bf16 operand
+ * rounding does not average out over so few elements)). */
 MUON_API muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds);
 
 /* Optional timing: `events` holds 2 * launches cudaEvent_t (as void*); each
@@ -197,10 +202,12 @@ MUON_API muon_status_t muon_plan_flops(muon_plan_t plan, double* gram, double* p
 MUON_API void muon_plan_destroy(muon_plan_t plan);
 
 /* ---------------------------------------------------------------- one-shot
- * Plan, execute and destroy in one call. The descriptor copy is issued on
- * `stream` from host memory that the call releases before returning (a
- * pageable copy, staged by the CUDA runtime), so these are not meant for
- * CUDA graph capture: capture muon_plan_execute instead. */
+ * Plan, execute and destroy in one call. The plan's descriptor tables reach
+ * the workspace as kernel arguments (at most 32 KB per launch; all-zero
+ * chunks as memsets), so no device work left pending by the call refers to
+ * the host memory it releases, and the call does not wait on the stream.
+ * A persistent plan (muon_plan_execute) saves the planning and this copy on
+ * every later call. */
 
 MUON_API muon_status_t muon_workspace_size(const muon_param_t* params, int count, muon_precision_t prec,
                                   size_t* bytes);

@@ -126,7 +126,7 @@ class _PlanBase:
     def launches(self):
         """Kinds of the kernels one execute launches (0 elementwise, 1 Gram,
         2 polynomial, 3 apply, 4 apply + update, 5 small-matrix kernel,
-        6 RMS reduction, 7 update pass, 8 mid-size kernel)."""
+        6 RMS reduction, 7 update pass, 8 mid-size kernel, 9 tiny fp32 kernel)."""
         lib = _lib.load()
         n = ctypes.c_int()
         _check(lib.muon_plan_launches(self._plan, ctypes.byref(n), None, 0), "launches")

@@ -123,9 +123,10 @@ struct muon_plan_s {
          ws_bytes = 0;
   std::vector<int32_t> small_mats;  // internal indices run by the small-matrix kernel
   std::vector<int32_t> mid_mats;    // internal indices run by the mid-size kernel
-  size_t off_mid = 0;
+  std::vector<int32_t> tiny_mats;   // internal indices run by the tiny fp32 kernel
+  size_t off_mid = 0, off_tiny = 0;
   std::vector<int> launch_kinds;    // 0 elementwise, 1 Gram, 2 Poly, 3 Apply, 4 ApplyLast, 5 small, 8 mid,
-                                    // 6 RMS reduction, 7 update pass (unit-RMS scale)
+                                    // 9 tiny, 6 RMS reduction, 7 update pass (unit-RMS scale)
   int scale_mode = MUON_SCALE_SHAPE;
   int sumsq_per_tile = 1;           // sum-of-squares slots per Apply tile (unit-RMS scale)
   size_t off_sumsq = 0, off_factor = 0;
@@ -135,6 +136,9 @@ struct muon_plan_s {
   size_t l2_batch_bytes = 0;
   std::vector<std::pair<int, int>> batches;  // internal matrix ranges [first, last)
   std::vector<uint8_t> blob;
+  // one-shot calls: the descriptor tables travel as kernel arguments, since
+  // the plan (and its host image) ends when the call returns
+  bool upload_by_value = false;
   void* uploaded_ws = nullptr;
   int uploaded_dev = -1;
   std::vector<void*> events;
@@ -224,6 +228,7 @@ void make_launch_list(muon_plan_s* p) {
   p->launch_kinds.assign(1, 0);
   if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
   if (!p->mid_mats.empty()) p->launch_kinds.push_back(8);
+  if (!p->tiny_mats.empty()) p->launch_kinds.push_back(9);
   if (p->stage_tiles[kApply] > 0) {
     for (const auto& bt : p->batches) {
       if (first_tile(p, bt.first, kApply) == first_tile(p, bt.second, kApply)) continue;
@@ -275,7 +280,11 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     gd.count = static_cast<int32_t>(members[g].size());
     gd.first_mat = static_cast<int32_t>(p->mats.size());
     double fl[kNumKinds] = {0, 0, 0};
-    gd.small = (tc && r <= kSmallMax && c <= kSmallMax) ? 1 : (tc && r <= kSmallMax && c <= kMidMaxC) ? 2 : 0;
+    gd.small = !tc                                   ? 0
+               : (r * c <= kTinyMaxElems)              ? 3
+               : (r <= kSmallMax && c <= kSmallMax)    ? 1
+               : (r <= kSmallMax && c <= kMidMaxC)     ? 2
+                                                       : 0;
     if (gd.small) {
       // one CTA per matrix, dense 128 x 128 products; count the useful FLOPs
       fl[kGram] = 2.0 * r * r * static_cast<double>(c);
@@ -324,6 +333,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
       if (md.O && rows16 && (reinterpret_cast<uintptr_t>(md.O) & 15) == 0) md.flags |= kMatOTma;
       if (gd.small == 1) p->small_mats.push_back(static_cast<int32_t>(p->mats.size()));
       if (gd.small == 2) p->mid_mats.push_back(static_cast<int32_t>(p->mats.size()));
+      if (gd.small == 3) p->tiny_mats.push_back(static_cast<int32_t>(p->mats.size()));
       md.ew_tile_begin = ew_total;
       md.ew_tiles = cdiv(md.n, kEwRows) * cdiv(md.m, kEwCols);
       ew_total += md.ew_tiles;
@@ -349,6 +359,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + p->small_mats.size() * sizeof(int32_t), 256);
   p->off_mid = off;
   off = align_up(off + p->mid_mats.size() * sizeof(int32_t), 256);
+  p->off_tiny = off;
+  off = align_up(off + p->tiny_mats.size() * sizeof(int32_t), 256);
   p->off_partial = off;
   off = align_up(off + static_cast<size_t>(ew_total) * sizeof(float), 256);
   p->off_counter = off;
@@ -400,6 +412,8 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
     std::memcpy(p->blob.data() + p->off_small, p->small_mats.data(), p->small_mats.size() * sizeof(int32_t));
   if (!p->mid_mats.empty())
     std::memcpy(p->blob.data() + p->off_mid, p->mid_mats.data(), p->mid_mats.size() * sizeof(int32_t));
+  if (!p->tiny_mats.empty())
+    std::memcpy(p->blob.data() + p->off_tiny, p->tiny_mats.data(), p->tiny_mats.size() * sizeof(int32_t));
   make_launch_list(p);
   auto* tile_mat = reinterpret_cast<int32_t*>(p->blob.data() + p->off_tile_mat);
   for (size_t k = 0; k < nm; ++k)
@@ -455,9 +469,12 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
         return MUON_ERR_CUDA;
     }
   }
-  if (cudaMemcpyAsync(ws, p->blob.data(), p->desc_bytes, cudaMemcpyHostToDevice, stream) !=
-      cudaSuccess)
+  if (p->upload_by_value) {
+    if (launch_blob_copy(ws, p->blob.data(), p->desc_bytes, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  } else if (cudaMemcpyAsync(ws, p->blob.data(), p->desc_bytes, cudaMemcpyHostToDevice, stream) !=
+             cudaSuccess) {
     return MUON_ERR_CUDA;
+  }
   p->uploaded_ws = ws;
   p->uploaded_dev = dev;
   return MUON_OK;
@@ -473,8 +490,8 @@ std::atomic<int> g_tracing{0};
 const char* kind_name(int kind) {
   static const char* names[] = {"muon:momentum+norm", "muon:gram", "muon:poly", "muon:apply",
                                 "muon:apply+update", "muon:small", "muon:rms", "muon:update",
-                                "muon:mid"};
-  return (kind >= 0 && kind < 9) ? names[kind] : "muon:?";
+                                "muon:mid", "muon:tiny"};
+  return (kind >= 0 && kind < 10) ? names[kind] : "muon:?";
 }
 
 // Slots come in pairs around launch slot / 2: timing events (when set) and
@@ -656,7 +673,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   const bool tc = plan->prec == MUON_NS_BF16;
   const int sms = g_num_sms[dev];
   int slot = 2;
-  if (!plan->small_mats.empty() || !plan->mid_mats.empty()) {
+  if (!plan->small_mats.empty() || !plan->mid_mats.empty() || !plan->tiny_mats.empty()) {
     SmallArgs sm{};
     sm.groups = groups;
     sm.mats = mats;
@@ -675,6 +692,9 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
     sm.scale_mode = plan->scale_mode;
     sm.diag = plan->mode == 0 ? plan->diag : nullptr;
     sm.wait_limit_ns = limit;
+    sm.mode = plan->mode;
+    sm.nesterov = ew.nesterov;
+    sm.mu = ew.mu;
     for (int k = 0; k < 3 * plan->steps; ++k) sm.abc[k] = plan->abc[k];
     if (sm.nsmall > 0) {
       const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 2LL * sms));
@@ -688,6 +708,14 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
       const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, static_cast<int64_t>(sms)));
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
       if (launch_mid(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
+    if (!plan->tiny_mats.empty()) {
+      sm.small_mats = reinterpret_cast<const int32_t*>(ws + plan->off_tiny);
+      sm.nsmall = static_cast<int64_t>(plan->tiny_mats.size());
+      const int grid = static_cast<int>(std::min<int64_t>(sm.nsmall, 3LL * sms));
+      if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      if (launch_tiny(sm, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
     }
   }
@@ -828,6 +856,7 @@ muon_status_t muon_step(const muon_param_t* params, int count, float lr, float m
   muon_plan_t p = nullptr;
   muon_status_t st = muon_plan_create(params, count, prec, sched, &p);
   if (st != MUON_OK) return st;
+  p->upload_by_value = true;
   muon_hyper_t h{lr, momentum, weight_decay, gamma, nesterov};
   st = muon_plan_execute(p, &h, workspace, workspace_bytes, stream);
   muon_plan_destroy(p);
@@ -851,6 +880,7 @@ muon_status_t ns_orthogonalize(const muon_ns_matrix_t* mats, int count,
   muon_plan_t p = nullptr;
   muon_status_t st = muon_plan_create_ns(mats, count, prec, sched, &p);
   if (st != MUON_OK) return st;
+  p->upload_by_value = true;
   st = muon_plan_execute(p, nullptr, workspace, workspace_bytes, stream);
   muon_plan_destroy(p);
   return st;
@@ -905,7 +935,26 @@ muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream) 
 
 namespace muon {
 
+void plan_upload_by_value(muon_plan_t plan) {
+  if (plan) plan->upload_by_value = true;
+}
+
 namespace {
+
+// One chunk of host bytes carried in the launch's parameter space (kernel
+// parameters may take up to 32764 bytes): the launch copies them to `dst`.
+constexpr int kBlobChunkWords = 2040;  // 32,640 bytes of 16-byte words
+struct BlobChunk {
+  uint4 data[kBlobChunkWords];
+  uint4* dst;
+  uint32_t words;
+};
+static_assert(sizeof(BlobChunk) <= 32764, "kernel parameter limit");
+
+__global__ void blob_copy_kernel(const __grid_constant__ BlobChunk c) {
+  for (uint32_t i = threadIdx.x; i < c.words; i += blockDim.x) c.dst[i] = c.data[i];
+}
+
 __global__ void wait_probe_kernel(const int* flag, int* err, unsigned long long limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint64_t it = 0; it < ptx::kSpinBackstop; ++it) {
@@ -916,6 +965,34 @@ __global__ void wait_probe_kernel(const int* flag, int* err, unsigned long long 
   atomicOr(err, kErrTimeout);
 }
 }  // namespace
+
+// Copy `bytes` (a multiple of 16; `dst` 16-byte aligned) from host memory to
+// the device in launches that carry the bytes as kernel arguments. Chunks of
+// zeros become memsets. Nothing on the device refers to `src` afterwards.
+cudaError_t launch_blob_copy(void* dst, const void* src, size_t bytes, cudaStream_t stream) {
+  if ((bytes & 15) != 0 || (reinterpret_cast<uintptr_t>(dst) & 15) != 0) return cudaErrorInvalidValue;
+  static thread_local BlobChunk chunk;  // 32 KB: kept off the stack
+  const auto* s = static_cast<const uint8_t*>(src);
+  constexpr size_t kChunkBytes = sizeof(chunk.data);
+  for (size_t off = 0; off < bytes; off += kChunkBytes) {
+    const size_t n = std::min(kChunkBytes, bytes - off);
+    bool zero = true;
+    for (size_t i = 0; i < n && zero; ++i) zero = s[off + i] == 0;
+    uint8_t* d = static_cast<uint8_t*>(dst) + off;
+    if (zero) {
+      const cudaError_t e = cudaMemsetAsync(d, 0, n, stream);
+      if (e != cudaSuccess) return e;
+      continue;
+    }
+    std::memcpy(chunk.data, s + off, n);
+    chunk.dst = reinterpret_cast<uint4*>(d);
+    chunk.words = static_cast<uint32_t>(n / 16);
+    blob_copy_kernel<<<1, 256, 0, stream>>>(chunk);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limit_ns,
                               cudaStream_t stream) {

@@ -27,6 +27,11 @@ cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream);
 // matrix (args.small_mats lists those matrices).
 cudaError_t launch_mid(const SmallArgs& args, int grid, cudaStream_t stream);
 
+// Matrices of at most kTinyMaxElems elements in the bf16 precision: every
+// step and the update with fp32 operands, one CTA per matrix (args.small_mats
+// lists those matrices).
+cudaError_t launch_tiny(const SmallArgs& args, int grid, cudaStream_t stream);
+
 // Unit-RMS update scale, grouped / fp32 path: per-matrix RMS of O' from the
 // last Apply's sums of squares, then W <- W (1 - lr wd) - lr (gamma / RMS) O'.
 cudaError_t launch_rms_reduce(const FinishArgs& args, cudaStream_t stream);
@@ -38,6 +43,11 @@ cudaError_t launch_stage_simt(StageKind kind, const StageArgs& args, int grid,
 
 // Dynamic shared memory the tcgen05 stage kernels need.
 size_t stage_tc_smem_bytes();
+
+// Copy `bytes` (a multiple of 16) of host memory to `dst` (16-byte aligned)
+// through kernel arguments, 32 KB per launch (all-zero chunks as memsets):
+// once the call returns, no pending device work refers to `src`.
+cudaError_t launch_blob_copy(void* dst, const void* src, size_t bytes, cudaStream_t stream);
 
 // Bounded wait on a host-visible word that nothing sets: used by the tests of
 // the timeout path. Sets the timeout bit of `err` when the limit passes.

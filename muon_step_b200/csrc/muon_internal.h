@@ -27,6 +27,10 @@ constexpr int kSmallMax = 128;
 // Matrices with min(n, m) <= kSmallMax < max(n, m) <= kMidMaxC run the whole
 // iteration in one 512-thread CTA with the iterate in shared memory.
 constexpr int kMidMaxC = 512;
+// In the bf16 precision, matrices of at most kTinyMaxElems elements run the
+// whole iteration with fp32 operands in one CTA (too few elements for bf16
+// operand rounding to average out over the Frobenius norm).
+constexpr int kTinyMaxElems = 4096;
 
 // fp32 validation tile shape.
 constexpr int kSBM = 64;
@@ -68,7 +72,8 @@ struct GroupDesc {
   int32_t ldc, ldr;      // leading dimensions (elements) of r x c and r x r buffers
   int32_t count;         // matrices in this group
   int32_t first_mat;     // internal index of the group's first matrix
-  int32_t small;         // 1: small-matrix kernel, 2: mid-size kernel (no stage tiles either way)
+  int32_t small;         // 1: small-matrix kernel, 2: mid-size kernel, 3: tiny fp32 kernel
+                         // (no stage tiles for any of them)
   int32_t pad0;
   int64_t xf_off[2];     // byte offsets in the workspace: fp32 iterate, ping-pong (fp32 mode)
   int64_t xb_off[2];     // bf16 iterate (bf16 mode: its high part, the MMA operand), ping-pong
@@ -152,6 +157,9 @@ struct SmallArgs {
   int32_t scale_mode;     // muon_scale_mode_t of the update
   uint64_t wait_limit_ns;
   float* diag;            // optional: diag[2 caller + 1] = RMS of the applied update O
+  int32_t mode;           // tiny kernel: 0 Muon step (N from M_t and G), 1 ns_orthogonalize (N = G)
+  int32_t nesterov;       // tiny kernel: N = mu M_t + G (else N = M_t)
+  float mu;               // tiny kernel: momentum coefficient
   float abc[kMaxSteps * 3];
 };
 

@@ -42,6 +42,12 @@ muon_status_t scratch_address(void** out) {
 
 }  // namespace
 
+namespace muon {
+// The plan's descriptor tables go to the device as kernel arguments (the plan
+// ends when this call returns). Defined with the planner.
+void plan_upload_by_value(muon_plan_t plan);
+}  // namespace muon
+
 extern "C" muon_status_t muon_step_static_scratch(const muon_param_t* params, int count, float lr,
                                                   float momentum, float weight_decay, float gamma,
                                                   int nesterov, const muon_ns_schedule_t* sched,
@@ -49,6 +55,7 @@ extern "C" muon_status_t muon_step_static_scratch(const muon_param_t* params, in
   muon_plan_t plan = nullptr;
   muon_status_t st = muon_plan_create(params, count, prec, sched, &plan);
   if (st != MUON_OK) return st;
+  muon::plan_upload_by_value(plan);
   size_t need = 0;
   st = muon_plan_workspace_size(plan, &need);
   if (st == MUON_OK && need > static_cast<size_t>(MUON_STATIC_SCRATCH_BYTES)) st = MUON_ERR_WORKSPACE;

@@ -14,19 +14,11 @@ from oracle import muon_oracle
 TOL_O = {"bf16": 2e-2, "fp32": 1e-4}   # O' against the oracle
 TOL_ELEMENTWISE = 1e-6                  # momentum, and the update given the GPU's own O'
 
-# Matrices with fewer elements than this are too small for the bf16 rounding
-# of the iterate operand to average out over the Frobenius norm: a CPU
-# emulation of the kernels' rounding (bf16 X, A, B; fp32 master iterate) on
-# 12,000 random Gaussian matrices of 2 to 64 elements reached 3.8e-2; with the
-# split bf16 high + low iterate, 3.0e-2 on 12,600 such matrices.
-TINY_ELEMENTS = 256
-TOL_O_TINY_BF16 = 5e-2
 
 
 def tol_o(precision, shape):
-    n, m = shape
-    if precision == "bf16" and n * m < TINY_ELEMENTS:
-        return TOL_O_TINY_BF16
+    """The O' bound for one matrix: 2e-2 in the bf16 precision, 1e-4 in fp32,
+    at every size."""
     return TOL_O[precision]
 
 
@@ -115,3 +107,26 @@ def check_ns(xs, precision="bf16", schedule=None, eps=1e-7):
 
 def all_within(errs):
     return all(e <= t for _, e, t in errs)
+
+
+def blockwise_oracle(Gb, Mb, hyper, schedule=None):
+    """O' of a permuted block-diagonal matrix P blockdiag(B_1 .. B_k) Q from
+    the float64 oracle, block by block: the blocks of G and M_prev are given
+    as [k, rows, cols] stacks (the same support). Every Newton-Schulz step
+    multiplies X by a polynomial in X X^T, which is block-diagonal under the
+    same row permutation when X is, and permutations commute with the
+    iteration; so O' is the oracle's iteration of each block divided by the
+    WHOLE matrix's norm, and zero off the blocks (pinned against the oracle's
+    whole-matrix step in tests/test_oracle_pins.py). Returns the blocks of O'
+    in the caller's orientation."""
+    sched = muon_oracle.HYBRID_SCHEDULE if schedule is None else schedule
+    mu = hyper["mu"]
+    Mt = muon_oracle.momentum(Mb, Gb, mu)
+    N = muon_oracle.nesterov(Mt, Gb, mu) if hyper["nesterov"] else Mt
+    fro = math.sqrt(float(np.sum(N * N)))
+    out = []
+    for Nj in N:
+        X, transposed = muon_oracle.orient(Nj)
+        O = muon_oracle.hybrid_newton_schulz(X / (fro + muon_oracle.DEFAULT_EPS), sched)
+        out.append(O.T if transposed else O)
+    return np.stack(out)

@@ -14,6 +14,7 @@ from muon_step_b200._lib import (MUON_ERR_INVALID_ARG, MUON_ERR_WORKSPACE, MUON_
                                  MUON_NS_FP32, MUON_OK, MuonHyper, MuonNsMatrix, MuonNsSchedule,
                                  MuonParam)
 
+TINY = 4096  # matrices of at most this many elements take the tiny fp32 kernel (bf16 precision)
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
                  if f.endswith(".h"))
@@ -135,17 +136,20 @@ def expected_workspace(shapes, prec):
     off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + ew * 4, 256)     # matrix of each elementwise tile
-    small = [(n, m) for n, m in shapes if prec == MUON_NS_BF16 and max(n, m) <= 128]
+    tc = prec == MUON_NS_BF16
+    small = [(n, m) for n, m in shapes if tc and n * m > TINY and max(n, m) <= 128]
     off = al(off + len(small) * 4, 256)  # small-matrix list
-    mid = [(n, m) for n, m in shapes if prec == MUON_NS_BF16 and min(n, m) <= 128 < max(n, m) <= 512]
+    mid = [(n, m) for n, m in shapes if tc and n * m > TINY and min(n, m) <= 128 < max(n, m) <= 512]
     off = al(off + len(mid) * 4, 256)  # mid-size list
+    tiny = [(n, m) for n, m in shapes if tc and n * m <= TINY]
+    off = al(off + len(tiny) * 4, 256)  # tiny-matrix list
     off = al(off + ew * 4, 256)     # partial sums
     off = al(off + nm * 4, 256)
     off = al(off + nm * 4, 256)
     # unit-RMS scale: sums of squares per Apply tile (16 slots on tensor cores), a factor per matrix
     if prec == MUON_NS_BF16:
         apply_tiles = sum(len(mem) * math.ceil(r / 256) * math.ceil(c / 256)
-                          for (r, c), mem in groups.items() if r > 128 or c > 512)
+                          for (r, c), mem in groups.items() if r * c > TINY and (r > 128 or c > 512))
         slots = 16
     else:
         apply_tiles = sum(len(mem) * math.ceil(r / 64) * math.ceil(c / 64) for (r, c), mem in groups.items())
@@ -194,19 +198,24 @@ def launch_list(lib, shapes, prec=MUON_NS_BF16):
 
 def test_launch_list(lib):
     grouped = [1, 2, 3] * 9 + [1, 2, 4]
-    # matrices up to 128 x 128 run in the one-CTA small-matrix kernel (kind 5)
-    assert launch_list(lib, [(64, 64)]) == [0, 5]
-    assert launch_list(lib, [(128, 128), (1, 1), (7, 100)]) == [0, 5]
+    # matrices of at most 4096 elements run with fp32 operands in the tiny-matrix kernel (kind 9)
+    assert launch_list(lib, [(64, 64)]) == [0, 9]
+    assert launch_list(lib, [(1, 1), (7, 100), (1, 4096), (4096, 1), (32, 128)]) == [0, 9]
+    # larger matrices up to 128 x 128 run in the one-CTA small-matrix kernel (kind 5)
+    assert launch_list(lib, [(65, 64), (128, 128)]) == [0, 5]
+    assert launch_list(lib, [(128, 128), (1, 1), (7, 100)]) == [0, 5, 9]
     assert launch_list(lib, [(300, 400)]) == [0] + grouped
     # min(n, m) <= 128 < max(n, m) <= 512: the one-CTA mid-size kernel (kind 8)
     assert launch_list(lib, [(129, 64)]) == [0, 8]
-    assert launch_list(lib, [(128, 512), (512, 100), (1, 129)]) == [0, 8]
+    assert launch_list(lib, [(128, 512), (512, 100), (1, 129)]) == [0, 8, 9]
     assert launch_list(lib, [(128, 513)]) == [0] + grouped
+    assert launch_list(lib, [(1, 4097)]) == [0] + grouped
     assert launch_list(lib, [(129, 129)]) == [0] + grouped
-    assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 5] + grouped
-    assert launch_list(lib, [(64, 64), (100, 300), (300, 400)]) == [0, 5, 8] + grouped
-    # the fp32 validation precision has no small-matrix kernel
+    assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 9] + grouped
+    assert launch_list(lib, [(65, 65), (100, 300), (300, 400)]) == [0, 5, 8] + grouped
+    # the fp32 validation precision runs every matrix on the grouped fp32 kernels
     assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + grouped
+    assert launch_list(lib, [(2, 3)], MUON_NS_FP32) == [0] + grouped
 
 
 def test_scale_modes_change_the_launch_list(lib):
@@ -227,10 +236,10 @@ def test_scale_modes_change_the_launch_list(lib):
     assert kinds_now() == shape
     assert lib.muon_plan_set_scale_mode(plan, 3) == MUON_ERR_INVALID_ARG
     lib.muon_plan_destroy(plan)
-    # small matrices only: the small-matrix kernel reduces on chip
-    st, plan = create(lib, [(64, 64)])
+    # small and tiny matrices only: their one-CTA kernels reduce on chip
+    st, plan = create(lib, [(64, 64), (128, 128)])
     assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
-    assert kinds_now() == [0, 5]
+    assert kinds_now() == [0, 5, 9]
     lib.muon_plan_destroy(plan)
     # diagnostics add one reduction after the fused last step (shape / none scale)
     st, plan = create(lib, [(64, 64), (300, 400)])
@@ -314,7 +323,7 @@ def test_shard_calls_validate_before_touching_a_device(lib):
 
 
 def test_l2_batching_repeats_the_stage_launches_per_batch(lib):
-    shapes = [(300, 400), (400, 300), (300, 400), (64, 64)]
+    shapes = [(300, 400), (400, 300), (300, 400), (100, 100)]
     st, plan = create(lib, shapes)
     assert st == MUON_OK
     cnt = ctypes.c_int()
@@ -366,10 +375,12 @@ if given is not None:
         lib.muon_plan_destroy(plan)
         assert n.value == expected_workspace(shapes, prec)
         tc = prec == MUON_NS_BF16
-        small = tc and any(max(a, b) <= 128 for a, b in shapes)
-        mid = tc and any(min(a, b) <= 128 < max(a, b) <= 512 for a, b in shapes)
-        large = any(not tc or not (min(a, b) <= 128 and max(a, b) <= 512) for a, b in shapes)
-        want = [0] + ([5] if small else []) + ([8] if mid else [])
+        tiny = tc and any(a * b <= TINY for a, b in shapes)
+        small = tc and any(a * b > TINY and max(a, b) <= 128 for a, b in shapes)
+        mid = tc and any(a * b > TINY and min(a, b) <= 128 < max(a, b) <= 512 for a, b in shapes)
+        large = any(not tc or (a * b > TINY and not (min(a, b) <= 128 and max(a, b) <= 512))
+                    for a, b in shapes)
+        want = [0] + ([5] if small else []) + ([8] if mid else []) + ([9] if tiny else [])
         if large:
             want += [1, 2, 3] * 9 + [1, 2, 4]
         assert launch_list(lib, shapes, prec) == want

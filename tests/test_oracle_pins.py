@@ -404,3 +404,33 @@ def test_none_mode_is_the_plain_direction_and_zero_stays_zero():
     for mode in ("unit_rms", "none"):
         W_z, _, _ = oracle.muon_step(W, Z, Z, lr=0.1, wd=0.01, scale_mode=mode)
         assert np.array_equal(W_z, W * (1 - 0.1 * 0.01))
+
+
+@pytest.mark.parametrize("n,m,br,bc", [(24, 96, 6, 24), (96, 24, 24, 6), (30, 30, 10, 10)])
+def test_permuted_block_diagonal_inputs_orthogonalise_blockwise(n, m, br, bc):
+    """For G and M_prev of the form P blockdiag(B_1 .. B_k) Q the oracle's O'
+    is exactly zero off the blocks, and on each block it is the iteration of
+    that block divided by the whole matrix's norm ([V4-book] §3: each step
+    multiplies by a polynomial in X X^T). The full-size GPU checks of the two
+    largest sweep bases rest on this."""
+    import workloads
+    from tests.parity import blockwise_oracle
+
+    wl, supports = workloads.make_block_permuted(n, m, 2, br, bc, device="cpu", seed=3)
+    h = wl.hyper
+    for i in range(wl.count):
+        W, G, M = (t[i].double().numpy() for t in (wl.W, wl.G, wl.M))
+        _, _, O = muon_oracle.muon_step(W, G, M, lr=h["lr"], mu=h["mu"], wd=h["wd"],
+                                        gamma=h["gamma"])
+        rows, cols = (t.numpy() for t in supports[i])
+        idx = (rows[:, :, None], cols[:, None, :])
+        off = O.copy()
+        off[idx] = 0.0
+        assert not off.any()
+        ref = blockwise_oracle(G[idx], M[idx], h)
+        assert np.max(np.abs(O[idx] - ref)) <= 1e-12 * np.max(np.abs(ref))
+        # the blocks share one normalisation: a block orthogonalised alone
+        # differs from it by far more than the agreement above
+        alone = muon_oracle.ns_orthogonalize(muon_oracle.nesterov(
+            muon_oracle.momentum(M[idx][0], G[idx][0], h["mu"]), G[idx][0], h["mu"]))
+        assert np.max(np.abs(alone - ref[0])) > 1e-7 * np.max(np.abs(ref))

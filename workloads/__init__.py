@@ -1,3 +1,4 @@
 """Seeded synthetic workloads shared by the tests, the oracle and the benchmark."""
 
-from .synth import HYPER, Workload, make, make_random, sweep_batch, sweep_shape  # noqa: F401
+from .synth import (HYPER, Workload, make, make_block_permuted, make_random,  # noqa: F401
+                    make_sweep_blocks, sweep_batch, sweep_block_shape, sweep_shape)

@@ -29,6 +29,11 @@ Workloads (shapes and distributions):
   random orthogonal factors when min(n, m) <= 512, else rank 64 plus noise
   N(0, (1e-4 / sqrt(max(n, m)))^2).
 
+``make_sweep_blocks`` gives a sweep point's shapes and batch with G and M_prev
+of the form P blockdiag(B_1, ..., B_k) Q (random row and column permutations P,
+Q; full-rank blocks of 512 rows with the sweep's spectrum), for element-wise
+checks at sizes where the oracle cannot take a whole matrix.
+
 Except for ``single_256x512``, whose M_prev is specified, M_prev is an
 independent draw of the workload's own gradient recipe, so that N keeps the
 intended spectrum. W is N(0, 0.02^2) everywhere. Hyper-parameters: lr 0.02,
@@ -284,6 +289,58 @@ def make_sweep(base, aspect, device="cpu", seed=5, count=None):
                                               g, device)
     return _finish(f"sweep_{base}_{aspect}", [((n, m), i) for i in range(count)],
                    {(n, m): (W, G, M)}, device)
+
+
+def sweep_block_shape(n, m, block=512):
+    """Block shape of the permuted block-diagonal sweep inputs: block x block
+    for a square matrix, block x 4 block (or 4 block x block) along the
+    aspect, so that min(n, m) / block blocks cover every row and column."""
+    if n == m:
+        return block, block
+    return (block, 4 * block) if n < m else (4 * block, block)
+
+
+def make_block_permuted(n, m, count, block_rows, block_cols, device="cpu", seed=6, name=None):
+    """`count` n x m matrices whose G and M_prev have the form
+    P blockdiag(B_1, ..., B_k) Q: k = n / block_rows = m / block_cols blocks
+    along the diagonal, P and Q random permutations of the rows and columns
+    (one pair per matrix, shared by its G and M_prev), every block a full-rank
+    block_rows x block_cols matrix with random orthogonal factors and singular
+    values geometric from 1 to 1e-4 (the sweep recipe for matrices of up to
+    512 rows). W ~ N(0, 0.02^2) as everywhere.
+
+    Returns (workload, supports): supports[i] = (rows, cols), int64 tensors of
+    shape [k, block_rows] and [k, block_cols], the row and column indices of
+    matrix i's blocks."""
+    if n % block_rows or m % block_cols or n // block_rows != m // block_cols:
+        raise ValueError("blocks must tile the diagonal")
+    k = n // block_rows
+    gw, gm, gg, gp = (_generator(device, 1000 * seed + j) for j in range(4))
+    W = _weights(count, n, m, gw, device)
+    G = torch.zeros((count, n, m), device=device, dtype=torch.float32)
+    M = torch.zeros_like(G)
+    sig = _geom(1.0, 1e-4, min(block_rows, block_cols), device)
+    supports = []
+    for i in range(count):
+        rows = torch.randperm(n, generator=gp, device=device).view(k, block_rows)
+        cols = torch.randperm(m, generator=gp, device=device).view(k, block_cols)
+        for dst, g in ((G, gg), (M, gm)):
+            blocks = spectrum_matrix(k, block_rows, block_cols, sig, g, device)
+            dst[i][rows[:, :, None], cols[:, None, :]] = blocks.to(torch.float32)
+        supports.append((rows, cols))
+    wl = _finish(name or f"blocks_{n}x{m}", [((n, m), i) for i in range(count)],
+                 {(n, m): (W, G, M)}, device)
+    return wl, supports
+
+
+def make_sweep_blocks(base, aspect, device="cpu", seed=6, count=None, block=512):
+    """A sweep point's shapes and batch with permuted block-diagonal G and
+    M_prev (make_block_permuted, blocks of sweep_block_shape)."""
+    n, m = sweep_shape(base, aspect)
+    count = sweep_batch(n, m) if count is None else count
+    br, bc = sweep_block_shape(n, m, block)
+    return make_block_permuted(n, m, count, br, bc, device, seed,
+                               name=f"sweep_blocks_{base}_{aspect}")
 
 
 def make(name, device="cpu", **kw):
