@@ -19,6 +19,7 @@ rank runs its own batch (independent problems, no data-path collective, weak
 scaling); value = FLOPs of all ranks / the slowest rank's time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --mode distributed   # one workload shared by the ranks (strong scaling)
     python bench.py --impl reference     # the float64 CPU oracle, timed on a sample
 """
 
@@ -52,6 +53,11 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", choices=["independent", "distributed"], default="independent",
+                    help="independent: every rank steps its own copy of the workload (weak "
+                         "scaling); distributed: the ranks share one workload, each stepping "
+                         "the matrices it owns, then one all-gather of the weights (strong "
+                         "scaling)")
     ap.add_argument("--config", default="dense_d4096")
     ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
     ap.add_argument("--no-e2e", action="store_true")
@@ -514,6 +520,100 @@ def _small_kwargs(config):
     return {}
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def run_distributed(args, rank, world, local_rank):
+    """Strong scaling over one workload ("Muon 优化器完全拆解…", section
+    "分布式工程"): every rank holds the whole workload (the same seeded W and G),
+    owns whole matrices balanced by Newton-Schulz FLOPs, steps them with the
+    single-GPU plan, and one all-gather hands the updated weights to every
+    rank. Timed per step: the owned step and the exchange, each with CUDA
+    events; value = the workload's FLOPs / the slowest rank's step time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import muon_step_b200 as ms
+    import workloads
+    from muon_step_b200.distributed import DistributedMuon
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs CUDA GPUs")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    timeout = datetime.timedelta(seconds=120)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timeout, device_id=dev)
+    else:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                                world_size=1, timeout=timeout, device_id=dev)
+    wl = workloads.make(args.config, device=dev)
+    h = wl.hyper
+    opt = DistributedMuon([(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)],
+                          precision=args.precision)
+    hyper = dict(lr=h["lr"], momentum=h["mu"], weight_decay=h["wd"], gamma=h["gamma"],
+                 nesterov=h["nesterov"])
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 0)):
+        opt.step(**hyper)
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    clocks = ClockSampler(local_rank, uuid=_nvml_uuid(local_rank))
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.window_begin()
+    t0.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        opt.compute(**hyper)
+        ev[k][1].record(stream)
+        opt.exchange()
+        ev[k][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.window_end()
+    dist.barrier()
+    clk = clocks.stop()
+    assert ms.sync_status() == 0
+    ms_max = max_over_ranks(t0.elapsed_time(t1), dev, world)
+    compute_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps, dev, world)
+    exchange_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps, dev, world)
+    flops = metric_flops(wl.shapes, len(HYBRID))
+    value = flops * args.steps / (ms_max / 1e3) / 1e12
+    owned = [len(o) for o in opt.owned]
+    launches = len(opt._plan.launches()) if getattr(opt, "_plan", None) is not None else 0
+    if world > 1:
+        launches += 4  # pack and unpack: a descriptor copy and the copy kernel each
+    if rank == 0:
+        xbytes = opt.exchange_bytes()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": args.precision, "data": "synthetic",
+            "config": {"workload": args.config, "mode": "distributed", "matrices": wl.count,
+                       "parallelism": f"owner-partitioned x{world}", "owned_per_rank": owned,
+                       "metric_flops_per_step": flops},
+            "compute_ms_per_step": compute_ms, "exchange_ms_per_step": exchange_ms,
+            "exchange": {"collective": "all_gather (NCCL, in place)", "bytes_in_per_rank": xbytes,
+                         "gbs_per_rank": (xbytes / (exchange_ms / 1e3) / 1e9) if exchange_ms > 0 else None},
+            "gpu_launches": launches * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    del opt
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -521,6 +621,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.mode == "distributed":
+        return run_distributed(args, rank, world, local_rank)
 
     import datetime
 

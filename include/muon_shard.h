@@ -21,12 +21,18 @@
  * operations in the same order, so a one-rank sharded step equals muon_step()
  * given the same orthogonalised direction.
  *
+ * muon_copy_segments is the gather / permute step of a grouped exchange: it
+ * moves every matrix's shards between a per-matrix layout and a rank-major
+ * one in one launch, so that each of the steps 1, 3 and 7 is one collective
+ * over one buffer instead of one per matrix.
+ *
  * Conventions are those of muon_step.h (caller-owned fp32 DEVICE arrays, no
  * device allocation, asynchronous on `stream`, argument errors returned
- * synchronously). The descriptor list is copied into `workspace`
- * (muon_shard_workspace_size bytes, 256-byte aligned) with cudaMemcpyAsync
- * from pageable host memory on every call, so these calls are not for graph
- * capture.
+ * synchronously). Each call writes its descriptor list into `workspace`
+ * (muon_shard_workspace_size bytes, 256-byte aligned) through kernel
+ * arguments before its kernel runs, so the workspace must not be shared by
+ * calls that run concurrently, and nothing refers to host memory after the
+ * call returns.
  */
 #ifndef MUON_SHARD_H
 #define MUON_SHARD_H
@@ -57,7 +63,14 @@ typedef struct {
   int64_t n, m;
 } muon_shard_update_t;
 
-/* Workspace bytes for a list of `count` shards (either kind). */
+/* One segment of a copy: dst[i] = src[i] for 0 <= i < numel (fp32). */
+typedef struct {
+  float* dst;
+  const float* src;
+  int64_t numel;
+} muon_segment_t;
+
+/* Workspace bytes for a list of `count` shards or segments (any kind). */
 MUON_API muon_status_t muon_shard_workspace_size(int count, size_t* bytes);
 
 MUON_API muon_status_t muon_shard_momentum(const muon_shard_momentum_t* shards, int count,
@@ -67,6 +80,13 @@ MUON_API muon_status_t muon_shard_momentum(const muon_shard_momentum_t* shards, 
 MUON_API muon_status_t muon_shard_update(const muon_shard_update_t* shards, int count, float lr,
                                          float weight_decay, float gamma, void* workspace,
                                          size_t workspace_bytes, void* stream);
+
+/* Copy every segment, one launch over all of them (HBM-bound: 8 bytes per
+ * element). Pointers need 4-byte alignment; a segment whose two pointers are
+ * 16-byte aligned moves 16 bytes per access. 0 <= numel <= 2^40. No
+ * destination may overlap another segment's destination or any source. */
+MUON_API muon_status_t muon_copy_segments(const muon_segment_t* segs, int count, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

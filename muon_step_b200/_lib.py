@@ -35,7 +35,7 @@ EXPORTS = (
     "muon_adamw_plan_create", "muon_adamw_plan_workspace_size", "muon_adamw_plan_execute",
     "muon_adamw_plan_numel", "muon_adamw_plan_destroy", "muon_adamw_workspace_size",
     "muon_adamw_step",
-    "muon_shard_workspace_size", "muon_shard_momentum", "muon_shard_update",
+    "muon_shard_workspace_size", "muon_shard_momentum", "muon_shard_update", "muon_copy_segments",
     "muon_plan_set_l2_batching", "muon_set_tracing",
 )
 
@@ -74,6 +74,10 @@ class ShardMomentum(ctypes.Structure):
 class ShardUpdate(ctypes.Structure):
     _fields_ = [("W", ctypes.c_void_p), ("O", ctypes.c_void_p), ("numel", ctypes.c_int64),
                 ("n", ctypes.c_int64), ("m", ctypes.c_int64)]
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("dst", ctypes.c_void_p), ("src", ctypes.c_void_p), ("numel", ctypes.c_int64)]
 
 
 class MuonHyper(ctypes.Structure):
@@ -123,6 +127,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                      vp, ctypes.c_size_t, vp]),
         "muon_shard_update": (st, [P(ShardUpdate), ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                    ctypes.c_float, vp, ctypes.c_size_t, vp]),
+        "muon_copy_segments": (st, [P(Segment), ctypes.c_int, vp, ctypes.c_size_t, vp]),
         "muon_workspace_size": (st, [P(MuonParam), ctypes.c_int, ctypes.c_int, P(ctypes.c_size_t)]),
         "muon_step": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                            ctypes.c_float, ctypes.c_int, P(MuonNsSchedule), ctypes.c_int, vp,

@@ -11,8 +11,9 @@ all-reduce), and:
 2. each rank runs the single-GPU step (muon_step_b200.MuonPlan) over the
    matrices it owns: momentum buffers of other ranks' matrices are not
    touched and may be omitted (ZeRO-1 style optimizer-state sharding);
-3. every owner broadcasts its updated weights as one packed buffer (NCCL over
-   NVLink between GPUs), so all ranks end the step with identical weights.
+3. one all-gather over equal, padded per-rank slots of one buffer (NCCL over
+   NVLink between GPUs) hands every owner's updated weights to every rank, so
+   all ranks end the step with identical weights.
 
 One process per GPU, torch.distributed for the plumbing.
 """
@@ -48,17 +49,60 @@ def partition(shapes: Sequence, world: int) -> list:
     return owner
 
 
+class SegmentCopier:
+    """One launch that copies a fixed list of (dst, src) fp32 tensor pairs:
+    the library's muon_copy_segments. ``prepare`` builds the descriptor list
+    once; the returned callable issues the copy on the current stream."""
+
+    def __init__(self, device):
+        from . import _lib
+        self._lib = _lib.load()
+        self.device = torch.device(device)
+
+    def prepare(self, pairs):
+        from ._lib import Segment
+        pairs = [(d, s) for d, s in pairs if d.numel()]
+        if not pairs:
+            return lambda: None
+        for d, s in pairs:
+            if d.device.type != "cuda" or s.device != d.device or d.numel() != s.numel() \
+                    or d.dtype != torch.float32 or s.dtype != torch.float32 \
+                    or not d.is_contiguous() or not s.is_contiguous():
+                raise ValueError("segments are contiguous fp32 CUDA tensors of equal size")
+        arr = (Segment * len(pairs))(*[Segment(d.data_ptr(), s.data_ptr(), d.numel()) for d, s in pairs])
+        nbytes = ctypes.c_size_t()
+        st = self._lib.muon_shard_workspace_size(len(pairs), ctypes.byref(nbytes))
+        if st != 0:
+            raise RuntimeError(f"muon_shard_workspace_size: status {st}")
+        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=self.device)
+        keep = list(pairs)  # the tensors must outlive the descriptor list
+
+        def run():
+            st = self._lib.muon_copy_segments(arr, len(keep), ws.data_ptr(), ws.numel(),
+                                              torch.cuda.current_stream().cuda_stream)
+            if st != 0:
+                raise RuntimeError(f"muon_copy_segments: status {st}")
+        return run
+
+
 class DistributedMuon:
     """Muon step over matrices shared by every rank of ``group``.
 
     params: list of (W, G, M) per matrix, identical shapes and order on every
     rank; M may be None on ranks that do not own the matrix. ``compute``
     replaces the per-rank single-GPU step (a callable taking the owned
-    indices and the hyper-parameters), e.g. for tests on CPU ranks.
+    indices and the hyper-parameters), and ``copier`` the segment copy (an
+    object with ``prepare(pairs) -> callable``), e.g. for tests on CPU ranks.
+
+    The exchange is one all-gather: every rank packs its updated weights into
+    its slot of one buffer of world equal slots (each as long as the largest
+    rank's share, a multiple of 4 elements), the slots are gathered in place
+    (NCCL), and every rank unpacks the other owners' weights. Packing and
+    unpacking are one segment-copy launch each.
     """
 
     def __init__(self, params: Sequence, group=None, precision="bf16", schedule=None,
-                 eps=None, compute: Optional[Callable] = None):
+                 eps=None, compute: Optional[Callable] = None, copier=None):
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
@@ -83,36 +127,54 @@ class DistributedMuon:
             self._plan, self._ws = plan, ws
         self._compute = compute
         W0 = self.params[0][0]
-        self._bufs = [torch.empty(sum(self.params[k][0].numel() for k in self.owned[r]),
-                                  dtype=W0.dtype, device=W0.device) for r in range(self.world)]
-
-    def _src(self, r):
-        return dist.get_global_rank(self.group, r) if self.group is not None else r
-
-    def step(self, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True):
-        hyper = dict(lr=lr, momentum=momentum, weight_decay=weight_decay, gamma=gamma,
-                     nesterov=nesterov)
-        mine = self.owned[self.rank]
-        self._compute(mine, hyper)
-        # pack this rank's updated weights
-        buf, off = self._bufs[self.rank], 0
-        for k in mine:
-            W = self.params[k][0]
-            buf[off:off + W.numel()].copy_(W.reshape(-1))
-            off += W.numel()
-        # every owner broadcasts, in rank order (the same sequence on every rank)
+        if not all(p[0].is_contiguous() for p in self.params):
+            raise ValueError("weights must be contiguous")
+        if copier is None:
+            if W0.device.type != "cuda":
+                raise ValueError("DistributedMuon needs a copier for tensors that are not on a GPU")
+            copier = SegmentCopier(W0.device)
+        share = [sum(self.params[k][0].numel() for k in self.owned[r]) for r in range(self.world)]
+        self.slot = -(-max(share) // 4) * 4  # elements per rank slot (16-byte multiples)
+        self._gather = torch.empty(self.world * self.slot, dtype=W0.dtype, device=W0.device)
+        pack, unpack = [], []
         for r in range(self.world):
-            if self._bufs[r].numel():
-                dist.broadcast(self._bufs[r], src=self._src(r), group=self.group)
-        # unpack the other owners' weights
-        for r in range(self.world):
-            if r == self.rank:
-                continue
-            off = 0
+            off = r * self.slot
             for k in self.owned[r]:
                 W = self.params[k][0]
-                W.copy_(self._bufs[r][off:off + W.numel()].view_as(W))
+                seg = self._gather[off:off + W.numel()]
+                if r == self.rank:
+                    pack.append((seg, W.reshape(-1)))
+                else:
+                    unpack.append((W.reshape(-1), seg))
                 off += W.numel()
+        self._pack = copier.prepare(pack)
+        self._unpack = copier.prepare(unpack)
+        self._in_place = dist.get_backend(group) == "nccl"
+
+    def step(self, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True):
+        self.compute(lr, momentum, weight_decay, gamma, nesterov)
+        self.exchange()
+
+    def compute(self, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True):
+        """The step of the matrices this rank owns (no communication)."""
+        hyper = dict(lr=lr, momentum=momentum, weight_decay=weight_decay, gamma=gamma,
+                     nesterov=nesterov)
+        self._compute(self.owned[self.rank], hyper)
+
+    def exchange_bytes(self):
+        """Bytes each rank receives per exchange (the other ranks' slots)."""
+        return 0 if self.world == 1 else (self.world - 1) * self.slot * self._gather.element_size()
+
+    def exchange(self):
+        """Hand every owner's updated weights to every rank: pack, one
+        all-gather, unpack (nothing with one rank)."""
+        if self.world == 1:
+            return
+        self._pack()
+        mine = self._gather[self.rank * self.slot:(self.rank + 1) * self.slot]
+        dist.all_gather_into_tensor(self._gather, mine if self._in_place else mine.clone(),
+                                    group=self.group)
+        self._unpack()
 
 
 # ---------------------------------------------------------------------------
@@ -127,7 +189,7 @@ def shard_size(numel: int, world: int) -> int:
 
 
 class _ShardKernels:
-    """The library's shard kernels and ns_orthogonalize (C ABI)."""
+    """The library's shard kernels, segment copy and ns_orthogonalize (C ABI)."""
 
     def __init__(self, n_items, device):
         from . import _lib
@@ -139,9 +201,13 @@ class _ShardKernels:
         self.ws = torch.empty(max(nbytes.value, 256), dtype=torch.uint8, device=device)
         self.ns_plan = None
         self.ns_ws = None
+        self._copier = SegmentCopier(device)
 
     def _stream(self):
         return torch.cuda.current_stream().cuda_stream
+
+    def prepare_copy(self, pairs):
+        return self._copier.prepare(pairs)
 
     def momentum(self, items, mu, nesterov):
         from ._lib import ShardMomentum
@@ -183,6 +249,13 @@ class ZeroMuon:
          (library kernel, one launch)
       7. all-gather of the weight shards -> the whole updated weights
 
+    Each exchange is one collective over one buffer: the exchanged buffers
+    are rank-major (rank r's shards of every matrix side by side, S elements
+    per rank), and one segment-copy launch moves the gradients into that
+    layout before step 1 and the gathered N and weights out of it after steps
+    3 and 7, into the per-matrix buffers that Newton-Schulz and the caller
+    read.
+
     Every rank computes the Newton-Schulz of every matrix, as the algorithm
     states (the whole matrix is gathered everywhere). Weights, gradients and
     the gathered buffers are owned here, flat and padded; ``weight(k)`` and
@@ -202,25 +275,43 @@ class ZeroMuon:
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.device = dev
         self.precision, self.schedule, self.eps = precision, schedule, eps
+        K = len(self.shapes)
         self.shard = [shard_size(n * m, self.world) for n, m in self.shapes]
+        self.offset = [sum(self.shard[:k]) for k in range(K)]  # within one rank's S elements
+        S = self.rank_elems = sum(self.shard)
         full = [s * self.world for s in self.shard]
         z = lambda k: torch.zeros(k, dtype=torch.float32, device=dev)
-        self._W = [z(f) for f in full]        # whole weights (padded); shard r is this rank's
-        self._G = [z(f) for f in full]        # local gradient (padded)
-        self._N = [z(f) for f in full]        # gathered Nesterov input (padded)
-        self._O = [z(f) for f in full]        # O' of the whole matrix (padded)
-        self.momentum_shards = [z(s) for s in self.shard]
-        self._g = [z(s) for s in self.shard]  # reduced gradient shard
-        self.kernels = kernels if kernels is not None else _ShardKernels(len(self.shapes), dev)
+        # per-matrix (matrix-major) buffers, padded; shard r of matrix k is [r s_k, (r + 1) s_k)
+        self._W = [z(f) for f in full]        # whole weights
+        self._G = [z(f) for f in full]        # local gradient
+        self._N = [z(f) for f in full]        # gathered Nesterov input
+        self._O = [z(f) for f in full]        # O' of the whole matrix
+        # rank-major exchange buffers: [rank][matrix][shard]
+        self._Grm = z(self.world * S)
+        self._Nrm = z(self.world * S)
+        self._Wrm = z(self.world * S)
+        self._g = z(S)                        # reduced gradient shards of this rank
+        self._mom = z(S)
+        self.momentum_shards = [self._mom[o:o + s] for o, s in zip(self.offset, self.shard)]
+        self.kernels = kernels if kernels is not None else _ShardKernels(K, dev)
         self._in_place = dist.get_backend(group) == "nccl"
+        rm = lambda buf, r, k: buf[r * S + self.offset[k]: r * S + self.offset[k] + self.shard[k]]
+        mm = lambda buf, r, k: buf[k][r * self.shard[k]:(r + 1) * self.shard[k]]
+        every = [(r, k) for r in range(self.world) for k in range(K)]
+        prep = self.kernels.prepare_copy
+        self._G_to_rm = prep([(rm(self._Grm, r, k), mm(self._G, r, k)) for r, k in every])
+        self._N_from_rm = prep([(mm(self._N, r, k), rm(self._Nrm, r, k)) for r, k in every])
+        self._W_from_rm = prep([(mm(self._W, r, k), rm(self._Wrm, r, k)) for r, k in every])
+        self._W_to_rm = prep([(rm(self._Wrm, r, k), mm(self._W, r, k)) for r, k in every])
+        self._mom_items = [(self.momentum_shards[k], self._g[self.offset[k]:self.offset[k] + self.shard[k]],
+                            rm(self._Nrm, self.rank, k)) for k in range(K)]
+        self._ns_pairs = [(self._view(self._N, k), self._view(self._O, k)) for k in range(K)]
+        self._upd_items = [(rm(self._Wrm, self.rank, k), mm(self._O, self.rank, k), self.shapes[k])
+                           for k in range(K)]
 
     def _view(self, buf, k):
         n, m = self.shapes[k]
         return buf[k][: n * m].view(n, m)
-
-    def _mine(self, buf, k):
-        s = self.shard[k]
-        return buf[k][self.rank * s:(self.rank + 1) * s]
 
     def weight(self, k):
         return self._view(self._W, k)
@@ -232,27 +323,26 @@ class ZeroMuon:
         """Copy the initial whole weights (identical on every rank)."""
         for k, W in enumerate(weights):
             self.weight(k).copy_(W)
+        self._W_to_rm()
+
+    def _gather(self, buf):
+        S = self.rank_elems
+        mine = buf[self.rank * S:(self.rank + 1) * S]
+        dist.all_gather_into_tensor(buf, mine if self._in_place else mine.clone(), group=self.group)
 
     def step(self, lr=0.02, momentum=0.95, weight_decay=0.1, gamma=0.2, nesterov=True):
-        K = len(self.shapes)
-        for k in range(K):  # 1. gradient shards
-            dist.reduce_scatter_tensor(self._g[k], self._G[k], group=self.group)
-        # 2. momentum on the shards, Nesterov shard written into its slot of N
-        self.kernels.momentum([(self.momentum_shards[k], self._g[k], self._mine(self._N, k))
-                               for k in range(K)], momentum, nesterov)
-        for k in range(K):  # 3. whole N on every rank
-            dist.all_gather_into_tensor(self._N[k], self._gather_src(self._N, k), group=self.group)
+        # 1. this rank's gradient shards, summed over the ranks
+        self._G_to_rm()
+        dist.reduce_scatter_tensor(self._g, self._Grm, group=self.group)
+        # 2. momentum on the shards; each Nesterov shard lands in this rank's slot
+        self.kernels.momentum(self._mom_items, momentum, nesterov)
+        # 3. the whole N on every rank
+        self._gather(self._Nrm)
+        self._N_from_rm()
         # 4. Newton-Schulz of every whole matrix
-        self.kernels.orthogonalize([(self._view(self._N, k), self._view(self._O, k)) for k in range(K)],
-                                   self.precision, self.schedule, self.eps)
+        self.kernels.orthogonalize(self._ns_pairs, self.precision, self.schedule, self.eps)
         # 5./6. update of this rank's weight shards
-        self.kernels.update([(self._mine(self._W, k), self._mine(self._O, k), self.shapes[k])
-                             for k in range(K)], lr, weight_decay, gamma)
-        for k in range(K):  # 7. whole updated weights
-            dist.all_gather_into_tensor(self._W[k], self._gather_src(self._W, k), group=self.group)
-
-    def _gather_src(self, buf, k):
-        # NCCL gathers in place (the input is the output's own slot); other
-        # backends get a copy of the slot
-        mine = self._mine(buf, k)
-        return mine if self._in_place else mine.clone()
+        self.kernels.update(self._upd_items, lr, weight_decay, gamma)
+        # 7. the whole updated weights
+        self._gather(self._Wrm)
+        self._W_from_rm()

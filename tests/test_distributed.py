@@ -105,7 +105,7 @@ def _oracle_compute(params):
 
 def _dist_step(rank, world, out_dir):
     params = [(W.clone(), G.clone(), M.clone()) for W, G, M in _inputs()]
-    opt = DistributedMuon(params, compute=_oracle_compute(params))
+    opt = DistributedMuon(params, compute=_oracle_compute(params), copier=TorchCopier())
     opt.step(**HYPER)
     opt.step(**HYPER)
     torch.save({"W": [p[0] for p in params], "M": [p[2] for p in params], "owner": opt.owner},
@@ -158,7 +158,22 @@ def _zero_kernels():
                 On = muon_oracle.rescale(O.double().numpy(), n, m, gamma)
                 W.copy_(torch.from_numpy(muon_oracle.decay_and_update(W.double().numpy(), On, lr, wd)))
 
+        def prepare_copy(self, pairs):
+            return TorchCopier().prepare(pairs)
+
     return K()
+
+
+class TorchCopier:
+    """CPU stand-in of the library's segment copy (host logic of the exchanges)."""
+
+    def prepare(self, pairs):
+        pairs = list(pairs)
+
+        def run():
+            for d, s in pairs:
+                d.copy_(s)
+        return run
 
 
 def _zero_step(rank, world, out_dir):

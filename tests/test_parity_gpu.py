@@ -418,3 +418,32 @@ def test_tiny_matrices_orthogonalize():
     xs = [torch.randn(n, m, generator=rng, device="cuda") for n, m in TINY]
     errs = check_ns(xs, "bf16")
     assert all(e <= TOL_O["fp32"] for _, e, _ in errs), errs
+
+
+def test_copy_segments_moves_every_segment():
+    """The segment copy of the grouped exchanges: ragged lengths, starts that
+    are not 16-byte aligned, an empty segment; bit-exact, nothing else written."""
+    import ctypes
+
+    from muon_step_b200 import _lib
+    from muon_step_b200._lib import Segment
+
+    lib = _lib.load()
+    g = torch.Generator(device="cuda").manual_seed(73)
+    src = torch.randn(100_003, generator=g, device="cuda")
+    dst = torch.full((100_003,), -1.0, device="cuda")
+    # (source offset, destination offset, elements); destinations do not overlap
+    cuts = [(0, 0, 4096), (5000, 4100, 17), (9, 20000, 30000), (70001, 50001, 1),
+            (1, 60000, 40000), (99999, 100002, 0), (4, 4096, 4)]
+    want = dst.clone()
+    for so, do, n in cuts:
+        want[do:do + n] = src[so:so + n]
+    segs = (Segment * len(cuts))(*[Segment(dst.data_ptr() + 4 * do, src.data_ptr() + 4 * so, n)
+                                    for so, do, n in cuts])
+    nbytes = ctypes.c_size_t()
+    assert lib.muon_shard_workspace_size(len(cuts), ctypes.byref(nbytes)) == 0
+    ws = torch.empty(nbytes.value, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.muon_copy_segments(segs, len(cuts), ws.data_ptr(), ws.numel(), stream) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(dst, want)
