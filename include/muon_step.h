@@ -114,8 +114,8 @@ typedef struct {
 
 /* How O' is scaled into the update O (W <- W (1 - lr wd) - lr O):
  *   SHAPE     O = O' sqrt(max(n, m)) gamma   ([V4-breakdown] Algorithm 1; default)
- *   UNIT_RMS  O = O' gamma / RMS(O')         ([V4-breakdown] "分布式工程": the
- *             Megatron-Bridge recipe's unit_rms_norm scale mode; O' = 0 gives O = 0)
+ *   UNIT_RMS  O = O' gamma / RMS(O')         ([V4-breakdown] "另一条路：开源生态干脆不分片":
+ *             the Megatron-Bridge recipe's unit_rms_norm scale mode; O' = 0 gives O = 0)
  *   NONE      O = O' gamma                   (the original Muon with gamma = 1) */
 typedef enum { MUON_SCALE_SHAPE = 0, MUON_SCALE_UNIT_RMS = 1, MUON_SCALE_NONE = 2 } muon_scale_mode_t;
 

@@ -1,6 +1,6 @@
 """Optimizer settings, including the Megatron-Bridge recipe keys.
 
-[V4-breakdown] "Muon 优化器完全拆解…", section "分布式工程", prints the
+[V4-breakdown] "Muon 优化器完全拆解…", section "另一条路：开源生态干脆不分片", prints the
 Megatron-Bridge DeepSeek-V4-Flash Muon recipe: muon_momentum,
 muon_use_nesterov, muon_scale_mode ("unit_rms_norm"), muon_fp32_matmul_prec,
 muon_num_ns_steps, muon_extra_scale_factor, muon_coefficient_type

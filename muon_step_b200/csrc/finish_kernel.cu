@@ -1,7 +1,7 @@
 // Update pass of the unit-RMS scale mode for matrices on the grouped (or
 // fp32) path.
 //
-// "Muon 优化器完全拆解…", section "分布式工程": the Megatron-Bridge recipe scales
+// "Muon 优化器完全拆解…", section "另一条路：开源生态干脆不分片": the Megatron-Bridge recipe scales
 // the update to unit RMS and then by an extra factor, O = gamma O' / RMS(O').
 // RMS(O') needs all of O' before any element of W can move, so here the last
 // Apply stage keeps O' in the iterate buffers and records sums of squares per

@@ -10,16 +10,17 @@ Sources (web pages on the method; cited by page title and section):
 
 * [V4-breakdown] "Muon 优化器完全拆解：矩阵级正交化更新如何撑起万亿 MoE 训练"
   (pinghaoyang.com.cn/aigc/posts/muon-optimizer-deepseek-v4/).
-  Section "V4 的完整更新公式，逐行拆解", Algorithm 1 "Muon Optimizer for
-  DeepSeek-V4" and the five numbered steps explained under it.
+  Section "V4 的完整更新公式，逐行拆解" (the update formula and its terms),
+  section "更新尺度：让 Muon 借用 AdamW 的超参" (the RMS rescale).
 * [V4-book] "Ch 06 · Muon — 矩阵参数的指南针" (DeepSeek-V4-book, chapter 6).
   §3 "Newton–Schulz：用 5 次 matmul 近似 polar" (the iteration),
   §4 "为什么 V4 要做 Hybrid 两段式 10 步" (the 8 + 2 schedule),
   §5 "完整算法" (the expanded Algorithm 1 "Muon Optimizer (V4 Hybrid)").
 
-Every step below is the plain definition, in float64, in the pages' order and
-notation. Matrix products use numpy's ``@`` (a library matmul) and nothing
-else: no blocking, fusion or reordering.
+Each function below is the plain mathematical definition of one term of the
+update, in float64 and in the pages' notation; ``muon_step`` composes them.
+Matrix products use numpy's ``@`` (a library matmul) and nothing else: no
+blocking, fusion or reordering.
 
 Readings where the pages leave a point open (each also listed in the design
 notes of the repository):
@@ -50,8 +51,8 @@ from __future__ import annotations
 
 import numpy as np
 
-# [V4-book] §4 and §5 Algorithm 1; [V4-breakdown] section "分布式工程"
-# (the Megatron-Bridge "deepseekv4" coefficient entry): eight aggressive
+# [V4-book] §4 and §5 Algorithm 1; [V4-breakdown] section
+# "另一条路：开源生态干脆不分片" (the Megatron-Bridge "deepseekv4" coefficient entry): eight aggressive
 # steps, then two standard Newton-Schulz steps.
 AGGRESSIVE_ABC = (3.4445, -4.7750, 2.0315)
 STANDARD_ABC = (2.0, -1.5, 0.5)
@@ -61,9 +62,9 @@ DEFAULT_EPS = 1e-7
 
 
 def momentum(M_prev: np.ndarray, G: np.ndarray, mu: float) -> np.ndarray:
-    """Momentum accumulation M_t = mu * M_{t-1} + G_t.
+    """Momentum accumulation M_t = mu * M_{t-1} + G_t (no dampening).
 
-    [V4-breakdown] Algorithm 1, "累积动量缓冲" step; [V4-book] §5 Algorithm 1.
+    [V4-breakdown] section "V4 的完整更新公式，逐行拆解"; [V4-book] §5.
     """
     return mu * M_prev + G
 
@@ -71,7 +72,7 @@ def momentum(M_prev: np.ndarray, G: np.ndarray, mu: float) -> np.ndarray:
 def nesterov(M: np.ndarray, G: np.ndarray, mu: float) -> np.ndarray:
     """Nesterov look-ahead N_t = mu * M_t + G_t (the input to orthogonalisation).
 
-    [V4-breakdown] Algorithm 1, "Nesterov 技巧" step; [V4-book] §5 Algorithm 1.
+    [V4-breakdown] section "V4 的完整更新公式，逐行拆解"; [V4-book] §5.
     """
     return mu * M + G
 
@@ -86,8 +87,8 @@ def orient(N: np.ndarray) -> tuple[np.ndarray, bool]:
 def frobenius_normalise(N: np.ndarray, eps: float = DEFAULT_EPS) -> np.ndarray:
     """X = N / (||N||_F + eps), which puts every singular value in [0, 1).
 
-    [V4-book] §5 Algorithm 1, the step that scales N into the convergence
-    region of the iteration.
+    [V4-book] §5: N is scaled into the region where the iteration of §3
+    converges.
     """
     fro = np.sqrt(np.sum(N * N))
     return N / (fro + eps)
@@ -96,15 +97,16 @@ def frobenius_normalise(N: np.ndarray, eps: float = DEFAULT_EPS) -> np.ndarray:
 def ns_step(X: np.ndarray, a: float, b: float, c: float) -> np.ndarray:
     """One Newton-Schulz step X <- a X + b (X X^T) X + c (X X^T)^2 X.
 
-    Written as the pages write it ([V4-book] §3 and §5 Algorithm 1):
-    three terms, each a product with the Gram matrix X X^T.
+    The quintic as [V4-book] §3 writes it: three terms, each a product with
+    the Gram matrix X X^T.
     """
     A = X @ X.T
     return a * X + b * (A @ X) + c * ((A @ A) @ X)
 
 
 def hybrid_newton_schulz(X0: np.ndarray, schedule=HYBRID_SCHEDULE) -> np.ndarray:
-    """Apply the schedule's steps in order ([V4-book] §4, §5 Algorithm 1)."""
+    """Compose the schedule's quintic steps, first to last ([V4-book] §4:
+    eight aggressive steps, then two standard ones, by default)."""
     X = X0
     for a, b, c in schedule:
         X = ns_step(X, a, b, c)
@@ -114,8 +116,7 @@ def hybrid_newton_schulz(X0: np.ndarray, schedule=HYBRID_SCHEDULE) -> np.ndarray
 def rescale(O_prime: np.ndarray, n: int, m: int, gamma: float) -> np.ndarray:
     """O = O' * sqrt(max(n, m)) * gamma.
 
-    [V4-breakdown] Algorithm 1, "缩放更新 RMS" step and section
-    "更新尺度：让 Muon 借用 AdamW 的超参"; [V4-book] §5 Algorithm 1.
+    [V4-breakdown] section "更新尺度：让 Muon 借用 AdamW 的超参"; [V4-book] §5.
     """
     return O_prime * (np.sqrt(float(max(n, m))) * gamma)
 
@@ -123,9 +124,10 @@ def rescale(O_prime: np.ndarray, n: int, m: int, gamma: float) -> np.ndarray:
 def rescale_unit_rms(O_prime: np.ndarray, gamma: float) -> np.ndarray:
     """O = gamma * O' / RMS(O'): the update normalised to unit RMS, then scaled.
 
-    [V4-breakdown] section "分布式工程", the Megatron-Bridge recipe's
-    muon_scale_mode "unit_rms_norm" with muon_extra_scale_factor gamma
-    ("把更新显式归一到单位 RMS 再乘 0.2"). A zero O' stays zero.
+    [V4-breakdown] section "另一条路：开源生态干脆不分片", the Megatron-Bridge
+    recipe's muon_scale_mode "unit_rms_norm" with muon_extra_scale_factor
+    gamma: the update is brought to unit RMS, then multiplied by the extra
+    factor (0.2 in that recipe). A zero O' stays zero.
     """
     rms = np.sqrt(np.mean(O_prime * O_prime))
     return O_prime * (gamma / rms) if rms > 0.0 else np.zeros_like(O_prime)
@@ -133,8 +135,8 @@ def rescale_unit_rms(O_prime: np.ndarray, gamma: float) -> np.ndarray:
 
 def rescale_none(O_prime: np.ndarray, gamma: float) -> np.ndarray:
     """O = gamma * O': no shape-dependent rescale, as in the original Muon
-    ([V4-breakdown] Algorithm 1 discussion: the original Muon had neither
-    weight decay nor the RMS rescale; gamma = 1 reproduces it)."""
+    ([V4-breakdown] section "V4 的完整更新公式，逐行拆解": the original Muon
+    had neither weight decay nor the RMS rescale; gamma = 1 reproduces it)."""
     return O_prime * gamma
 
 
@@ -144,7 +146,7 @@ SCALE_MODES = ("shape", "unit_rms", "none")
 def decay_and_update(W: np.ndarray, O: np.ndarray, lr: float, wd: float) -> np.ndarray:
     """Decoupled weight decay and step: W_t = W_{t-1} (1 - lr*wd) - lr * O_t.
 
-    [V4-breakdown] Algorithm 1, "权重衰减 + 更新" step; [V4-book] §5 Algorithm 1.
+    [V4-breakdown] section "V4 的完整更新公式，逐行拆解"; [V4-book] §5.
     """
     return W * (1.0 - lr * wd) - lr * O
 
@@ -160,12 +162,16 @@ def ns_orthogonalize(X: np.ndarray, schedule=HYBRID_SCHEDULE,
 
 def muon_step(W, G, M_prev, lr=0.02, mu=0.95, wd=0.1, gamma=0.2,
               nesterov_on=True, schedule=HYBRID_SCHEDULE, eps=DEFAULT_EPS, scale_mode="shape"):
-    """One Muon step for one n x m matrix, all in float64.
+    """One Muon step for one n x m matrix, all in float64:
 
-    Returns (W_t, M_t, O'_t) where O'_t is the orthogonalised direction before
-    the RMS rescale, in W's orientation. Follows [V4-breakdown] Algorithm 1 and
-    [V4-book] §5 Algorithm 1 step by step. With ``nesterov_on`` false the
-    orthogonaliser's input is M_t itself (the original Muon). ``scale_mode``
+        M_t = mu M_{t-1} + G_t,   N_t = mu M_t + G_t,
+        O'_t = NS(N_t / (||N_t||_F + eps)),
+        W_t = W_{t-1} (1 - lr wd) - lr * scale(O'_t),
+
+    the composition of the definitions above. Returns (W_t, M_t, O'_t) where
+    O'_t is the orthogonalised direction before the RMS rescale, in W's
+    orientation. With ``nesterov_on`` false the orthogonaliser's input is M_t
+    itself (the original Muon). ``scale_mode``
     picks the update's scale: "shape" (sqrt(max(n, m)) gamma, the default),
     "unit_rms" (gamma / RMS(O')) or "none" (gamma).
     """

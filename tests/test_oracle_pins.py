@@ -379,10 +379,11 @@ def test_planted_schedule_mistakes_are_caught(golden_dir, monkeypatch):
 # ----------------------------------------------------------------------------
 
 def test_unit_rms_mode_has_rms_gamma_and_matches_shape_mode():
-    """unit_rms_norm: RMS(O) = gamma exactly; in theory equal to the shape
-    rescale because RMS(O') ~ sqrt(1 / max(n, m)) ("Muon 优化器完全拆解…",
-    section "分布式工程": "两者在理论上等价"), so on well-conditioned inputs
-    the two agree within the band."""
+    """unit_rms_norm: RMS(O) = gamma exactly. The page calls it equivalent in
+    theory to the shape rescale, since the RMS of an orthogonalised update is
+    close to sqrt(1 / max(n, m)) ("Muon 优化器完全拆解…", section
+    "另一条路：开源生态干脆不分片"), so on well-conditioned inputs the two agree
+    within the band."""
     rng = np.random.default_rng(31)
     for n, m in [(48, 48), (32, 96), (96, 32)]:
         N = matrix_with_spectrum(rng, n, m, rng.uniform(0.7, 1.2, min(n, m)))
