@@ -62,6 +62,10 @@ def parse_args():
     ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
+    ap.add_argument("--stagewise", action="store_true",
+                    help="one launch per Newton-Schulz stage instead of the chained launch")
+    ap.add_argument("--chain-window", type=int, default=0,
+                    help="matrices the chained launch keeps in flight (0: from the tile counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
@@ -158,11 +162,20 @@ def dominant_roofline(kinds, per_kind_ms, shapes, peaks, precision="bf16", ns_st
     stage = "stage_tc_kernel" if precision == "bf16" else "stage_simt_kernel"
     names = {0: "ew_kernel", 1: f"{stage}<Gram>", 2: f"{stage}<Poly>", 3: f"{stage}<Apply>",
              4: f"{stage}<ApplyLast>", 5: "ns_small_kernel", 8: "ns_mid_kernel",
-             9: "ns_tiny_kernel", 6: "rms_reduce_kernel", 7: "finish_kernel"}
+             9: "ns_tiny_kernel", 6: "rms_reduce_kernel", 7: "finish_kernel",
+             10: "stage_chain_kernel"}
     grouped = [(n, m) for n, m in shapes if one_cta_kind(n, m, precision) is None]
     if dom in (1, 2, 3, 4):
         flops = executed_stage_flops(dom, grouped, precision)
         nbytes = stage_bytes(dom, grouped, precision)
+    elif dom == 10:
+        # every Gram, Poly and Apply stage but the last Apply (fused with the
+        # update, its own launch); bytes as if each stage read its operands
+        # and wrote its results through HBM
+        per = {k: (executed_stage_flops(k, grouped, precision), stage_bytes(k, grouped, precision))
+               for k in (1, 2, 3)}
+        flops = ns_steps * (per[1][0] + per[2][0] + per[3][0]) - per[3][0]
+        nbytes = ns_steps * (per[1][1] + per[2][1] + per[3][1]) - per[3][1]
     elif dom in (5, 8, 9):
         mine = [(n, m) for n, m in shapes if one_cta_kind(n, m, precision) == dom]
         flops = sum(ns_steps * (4.0 * min(n, m) ** 2 * max(n, m) + 2.0 * min(n, m) ** 3)
@@ -651,6 +664,7 @@ def main():
     h = wl.hyper
     params = [(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)]
     plan = ms.MuonPlan(params, precision=args.precision)
+    plan.set_chaining(not args.stagewise, args.chain_window)
     ws = plan.alloc_workspace()
     kinds = plan.launches()
     ns_steps = len(HYBRID)
@@ -822,7 +836,7 @@ def main():
 
     if rank == 0:
         names = {0: "elementwise", 1: "gram", 2: "poly", 3: "apply", 4: "apply_update", 5: "small",
-                 6: "rms_reduce", 7: "update", 8: "mid", 9: "tiny"}
+                 6: "rms_reduce", 7: "update", 8: "mid", 9: "tiny", 10: "chain"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -843,6 +857,7 @@ def main():
             "executed_tflops": executed,
             "gpu_launches": len(kinds) * args.steps,
             "cuda_graph": graph is not None,
+            "chained": 10 in kinds,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -167,6 +167,18 @@ MUON_API muon_status_t muon_plan_set_diagnostics(muon_plan_t plan, float* out);
  * not change. Timing events must be set again afterwards. */
 MUON_API muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes);
 
+/* How later executes launch the Newton-Schulz stages in the bf16 precision
+ * (without L2 batching). on = 1 (the default): every Gram, Poly and Apply
+ * stage of the schedule in one persistent launch, then the last Apply fused
+ * with the update. Its CTA pairs take the tiles of a host-built list in
+ * order; a tile waits (bounded) until the earlier stages of its own matrix
+ * have finished, signalled through per-matrix counters in the workspace. The
+ * list keeps `window` matrices in flight at a time (0: chosen from the tile
+ * counts), so their buffers can stay in L2 from one stage to the next.
+ * on = 0: one launch per stage and step. Both give bit-identical results.
+ * Timing events must be set again afterwards. */
+MUON_API muon_status_t muon_plan_set_chaining(muon_plan_t plan, int on, int window);
+
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */
 MUON_API muon_status_t muon_plan_workspace_size(muon_plan_t plan, size_t* bytes);
 
@@ -186,7 +198,8 @@ MUON_API muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* h
  * (all steps and the update of matrices with min(n, m) <= 128 < max(n, m)
  * <= 512), 9 tiny-matrix kernel (bf16 precision only: matrices of at most
  * 4096 elements run every step with fp32 operands, since bf16 operand
- * rounding does not average out over so few elements)). */
+ * rounding does not average out over so few elements), 10 chained launch of
+ * every Newton-Schulz stage (see muon_plan_set_chaining)). */
 MUON_API muon_status_t muon_plan_launches(muon_plan_t plan, int* count, int* kinds, int max_kinds);
 
 /* Optional timing: `events` holds 2 * launches cudaEvent_t (as void*); each
@@ -250,6 +263,14 @@ MUON_API void muon_set_wait_limit_ns(uint64_t ns);
  * `limit_ns`. If the limit passes, the device error word gets the timeout
  * bit, which muon_sync_status() then reports. */
 MUON_API muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream);
+
+/* Test of the chained launch's dependency wait (muon_plan_set_chaining): one
+ * thread waits, as a chained tile does, until the DEVICE word `counter`
+ * (acquire loads) reaches `target`, for at most `limit_ns`. If the limit
+ * passes, the device error word gets the timeout bit, which
+ * muon_sync_status() then reports. */
+MUON_API muon_status_t muon_dep_wait_probe(const uint32_t* counter, uint32_t target,
+                                           uint64_t limit_ns, void* stream);
 
 /* ---------------------------------------------------------------- no allocation
  * The pages describe no counterpart of this entry point; it serves callers

@@ -123,10 +123,19 @@ class _PlanBase:
         device = self.device if device is None else device
         return torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8, device=device)
 
+    def set_chaining(self, on: bool = True, window: int = 0):
+        """Run every Newton-Schulz stage in one chained launch (on, the
+        default) or one launch per stage and step (off); `window` is the number
+        of matrices the chained launch keeps in flight (0: from the tile
+        counts). Results are bit-identical; timing events must be set again."""
+        _check(_lib.load().muon_plan_set_chaining(self._plan, 1 if on else 0, int(window)),
+               "muon_plan_set_chaining")
+
     def launches(self):
         """Kinds of the kernels one execute launches (0 elementwise, 1 Gram,
         2 polynomial, 3 apply, 4 apply + update, 5 small-matrix kernel,
-        6 RMS reduction, 7 update pass, 8 mid-size kernel, 9 tiny fp32 kernel)."""
+        6 RMS reduction, 7 update pass, 8 mid-size kernel, 9 tiny fp32 kernel,
+        10 chained Newton-Schulz stages)."""
         lib = _lib.load()
         n = ctypes.c_int()
         _check(lib.muon_plan_launches(self._plan, ctypes.byref(n), None, 0), "launches")
@@ -461,3 +470,13 @@ def wait_probe(flag: torch.Tensor, limit_ns: int, stream=None):
         raise TypeError("flag must be an int32 CUDA tensor")
     _check(_lib.load().muon_wait_probe(flag.data_ptr(), int(limit_ns), _stream_ptr(stream)),
            "muon_wait_probe")
+
+
+def dep_wait_probe(counter: torch.Tensor, target: int, limit_ns: int, stream=None):
+    """Launch the chained launch's dependency wait on ``counter`` (int32 CUDA
+    tensor, read as unsigned) until it reaches ``target``, bounded by
+    ``limit_ns``."""
+    if counter.dtype != torch.int32 or counter.device.type != "cuda":
+        raise TypeError("counter must be an int32 CUDA tensor")
+    _check(_lib.load().muon_dep_wait_probe(counter.data_ptr(), int(target), int(limit_ns),
+                                           _stream_ptr(stream)), "muon_dep_wait_probe")

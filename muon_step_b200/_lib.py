@@ -36,7 +36,8 @@ EXPORTS = (
     "muon_adamw_plan_numel", "muon_adamw_plan_destroy", "muon_adamw_workspace_size",
     "muon_adamw_step",
     "muon_shard_workspace_size", "muon_shard_momentum", "muon_shard_update", "muon_copy_segments",
-    "muon_plan_set_l2_batching", "muon_set_tracing",
+    "muon_plan_set_l2_batching", "muon_set_tracing", "muon_plan_set_chaining",
+    "muon_dep_wait_probe",
 )
 
 
@@ -113,6 +114,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_plan_set_scale_mode": (st, [vp, ctypes.c_int]),
         "muon_plan_set_diagnostics": (st, [vp, vp]),
         "muon_plan_set_l2_batching": (st, [vp, ctypes.c_size_t]),
+        "muon_plan_set_chaining": (st, [vp, ctypes.c_int, ctypes.c_int]),
         "muon_set_tracing": (None, [ctypes.c_int]),
         "muon_adamw_plan_create": (st, [P(AdamwParam), ctypes.c_int, P(vp)]),
         "muon_adamw_plan_workspace_size": (st, [vp, P(ctypes.c_size_t)]),
@@ -140,6 +142,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "muon_abi_version": (ctypes.c_int, []),
         "muon_set_wait_limit_ns": (None, [ctypes.c_uint64]),
         "muon_wait_probe": (st, [vp, ctypes.c_uint64, vp]),
+        "muon_dep_wait_probe": (st, [vp, ctypes.c_uint32, ctypes.c_uint64, vp]),
         "muon_step_static_scratch": (st, [P(MuonParam), ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                           ctypes.c_float, ctypes.c_float, ctypes.c_int,
                                           P(MuonNsSchedule), ctypes.c_int, vp]),

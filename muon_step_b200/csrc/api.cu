@@ -37,6 +37,7 @@ std::mutex g_mutex;
 int* g_err_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
+int g_chain_pairs[kMaxDevices] = {};  // CTA pairs of the chained launch resident at once
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};  // set from any host thread
 
 // Per-device setup: the error word's device address and the SM count.
@@ -51,6 +52,11 @@ muon_status_t device_setup(int* dev_out) {
       return MUON_ERR_CUDA;
     g_cc_major[dev] = major;
     g_num_sms[dev] = sms;
+    if (major == 10) {
+      int pairs = 0;
+      if (chain_max_pairs(&pairs) != cudaSuccess) return MUON_ERR_CUDA;
+      g_chain_pairs[dev] = pairs;
+    }
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return MUON_ERR_CUDA;
     g_err_ptr[dev] = static_cast<int*>(p);
@@ -135,6 +141,12 @@ struct muon_plan_s {
   // matrices whose Newton-Schulz working set fits the budget (0: one batch)
   size_t l2_batch_bytes = 0;
   std::vector<std::pair<int, int>> batches;  // internal matrix ranges [first, last)
+  // chained launch of the Newton-Schulz stages (bf16, one pass): the tile
+  // list and the per-matrix dependency counters live in the descriptor region
+  bool chain_on = true;
+  int chain_window = 0;             // matrices in flight (0: from the tile counts)
+  int64_t chain_len = 0;            // tiles of every stage of every grouped matrix
+  size_t off_chain = 0, off_dep = 0;
   std::vector<uint8_t> blob;
   // one-shot calls: the descriptor tables travel as kernel arguments, since
   // the plan (and its host image) ends when the call returns
@@ -221,6 +233,11 @@ bool wide_epilogue(const muon_plan_s* p, const std::pair<int, int>& bt, int kind
   return tiles > 0.0 && ksum <= kmax * tiles;
 }
 
+// Whether the stages run as one chained launch (bf16, no L2 batching).
+bool chained(const muon_plan_s* p) {
+  return p->chain_on && p->prec == MUON_NS_BF16 && p->l2_batch_bytes == 0 && p->stage_tiles[kApply] > 0;
+}
+
 // The launch list of one execute (depends on the scale mode and the batches).
 void make_launch_list(muon_plan_s* p) {
   const bool unit = p->scale_mode == MUON_SCALE_UNIT_RMS;
@@ -229,6 +246,19 @@ void make_launch_list(muon_plan_s* p) {
   if (!p->small_mats.empty()) p->launch_kinds.push_back(5);
   if (!p->mid_mats.empty()) p->launch_kinds.push_back(8);
   if (!p->tiny_mats.empty()) p->launch_kinds.push_back(9);
+  if (chained(p)) {
+    // every stage in one launch; the last Apply fused with the update runs
+    // after it (in the unit-RMS mode the chain holds the last Apply too)
+    p->launch_kinds.push_back(10);
+    if (unit) {
+      p->launch_kinds.push_back(6);
+      p->launch_kinds.push_back(7);
+    } else {
+      p->launch_kinds.push_back(4);
+      if (p->diag) p->launch_kinds.push_back(6);
+    }
+    return;
+  }
   if (p->stage_tiles[kApply] > 0) {
     for (const auto& bt : p->batches) {
       if (first_tile(p, bt.first, kApply) == first_tile(p, bt.second, kApply)) continue;
@@ -373,6 +403,19 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   off = align_up(off + static_cast<size_t>(p->stage_tiles[kApply]) * p->sumsq_per_tile * sizeof(float), 256);
   p->off_factor = off;
   off = align_up(off + nm * sizeof(float), 256);
+  // chained launch: the tile list (every stage of every step of every grouped
+  // matrix) and one dependency counter per matrix
+  p->chain_len = 0;
+  if (tc)
+    for (const auto& md : p->mats) {
+      const GroupDesc& gd = p->groups[md.group];
+      p->chain_len += static_cast<int64_t>(p->steps) *
+                      (gd.tiles_per_mat[kGram] + gd.tiles_per_mat[kPoly] + gd.tiles_per_mat[kApply]);
+    }
+  p->off_chain = off;
+  off = align_up(off + static_cast<size_t>(p->chain_len) * sizeof(ChainTile), 256);
+  p->off_dep = off;
+  off = align_up(off + (tc ? nm * sizeof(unsigned) : 0), 256);
   p->desc_bytes = off;
   off = align_up(off, 1024);
   for (auto& gd : p->groups) {
@@ -430,7 +473,52 @@ bool valid_shape(int64_t n, int64_t m) {
   return n >= 1 && m >= 1 && n <= kMaxDim && m <= kMaxDim;
 }
 
+// The chained launch's tile list: a window of W matrices in flight, in
+// rounds; each round lists the next stage of every matrix in the window (all
+// its tiles), and a matrix that has finished every stage leaves the window
+// for the next one. A stage of a matrix is listed one round after the stage
+// it depends on, with the other matrices' tiles in between, so CTA pairs that
+// reach it seldom wait; the window's buffers are the working set that stays
+// in L2. W defaults to the number of matrices whose average stage gives
+// every CTA pair two tiles per round.
+void build_chain(const muon_plan_s* p, int npairs, ChainTile* out) {
+  std::vector<int> mats;
+  double stage_tiles = 0.0;
+  for (size_t i = 0; i < p->mats.size(); ++i) {
+    const GroupDesc& gd = p->groups[p->mats[i].group];
+    const int64_t per_step = gd.tiles_per_mat[kGram] + gd.tiles_per_mat[kPoly] + gd.tiles_per_mat[kApply];
+    if (per_step == 0) continue;
+    mats.push_back(static_cast<int>(i));
+    stage_tiles += per_step / 3.0;
+  }
+  if (mats.empty()) return;
+  int window = p->chain_window;
+  if (window <= 0) {
+    const double mean = stage_tiles / static_cast<double>(mats.size());
+    window = static_cast<int>(std::ceil(2.0 * std::max(npairs, 1) / std::max(mean, 1.0)));
+  }
+  window = std::max(1, std::min<int>(window, static_cast<int>(mats.size())));
+  const int nstages = 3 * p->steps;
+  std::vector<std::pair<int, int>> act;  // (matrix, next stage)
+  size_t next = 0;
+  int64_t k = 0;
+  while (next < mats.size() || !act.empty()) {
+    while (static_cast<int>(act.size()) < window && next < mats.size()) act.emplace_back(mats[next++], 0);
+    for (auto& x : act) {
+      const GroupDesc& gd = p->groups[p->mats[x.first].group];
+      const int kind = x.second % 3;
+      for (int64_t u = 0; u < gd.tiles_per_mat[kind]; ++u)
+        out[k++] = ChainTile{x.first, x.second, static_cast<int32_t>(u), 0};
+      ++x.second;
+    }
+    act.erase(std::remove_if(act.begin(), act.end(), [&](const std::pair<int, int>& x) { return x.second == nstages; }),
+              act.end());
+  }
+}
+
 muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
+  if (p->chain_len > 0)
+    build_chain(p, g_chain_pairs[dev], reinterpret_cast<ChainTile*>(p->blob.data() + p->off_chain));
   if (p->prec == MUON_NS_BF16) {
     char* base = static_cast<char*>(ws);
     auto* maps = reinterpret_cast<CUtensorMap*>(p->blob.data() + p->off_tmaps);
@@ -666,6 +754,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   ew.mu = plan->mode == 0 ? hyper->momentum : 0.f;
   ew.eps = plan->eps;
   ew.diag = plan->mode == 0 ? plan->diag : nullptr;
+  ew.dep = chained(plan) ? reinterpret_cast<unsigned*>(ws + plan->off_dep) : nullptr;
   if ((st = record(plan, 0, stream)) != MUON_OK) return st;
   if (launch_elementwise(ew, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if ((st = record(plan, 1, stream)) != MUON_OK) return st;
@@ -722,56 +811,95 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   if (plan->stage_tiles[kApply] == 0) return MUON_OK;
   const bool unit = plan->scale_mode == MUON_SCALE_UNIT_RMS;
   const bool diag = plan->mode == 0 && plan->diag != nullptr;
-  // one pass of every step per batch: a batch's buffers stay in L2 across its
-  // 3 x steps launches when the batch fits
-  for (const auto& bt : plan->batches)
-  for (int k = 0; k < plan->steps; ++k) {
-    if (first_tile(plan, bt.first, kApply) == first_tile(plan, bt.second, kApply)) break;
-    for (int kind = 0; kind < kNumKinds; ++kind) {
-      StageArgs sa{};
-      sa.groups = groups;
-      sa.mats = mats;
-      sa.tmaps = ws + plan->off_tmaps;
-      sa.mat_tmaps = ws + plan->off_mat_tmaps;
-      sa.ws = ws;
-      sa.scale = scale;
-      sa.err = err;
-      sa.tile_begin = first_tile(plan, bt.first, kind);
-      sa.total_tiles = first_tile(plan, bt.second, kind);
-      sa.ngroups = static_cast<int32_t>(plan->groups.size());
-      const bool last = k == plan->steps - 1;
-      sa.first = k == 0;
-      // unit-RMS scale: the last Apply keeps O' and its sums of squares; the
-      // update comes after the per-matrix reduction. Diagnostics: the fused
-      // last step records the sums too.
-      sa.last = last && !unit;
-      sa.scale_mode = plan->scale_mode;
-      if ((unit || diag) && last && kind == kApply) {
-        sa.sumsq_per_tile = plan->sumsq_per_tile;
-        sa.sumsq = reinterpret_cast<float*>(ws + plan->off_sumsq);
-      }
-      sa.xsrc = k & 1;
-      sa.a = plan->abc[3 * k];
-      sa.b = plan->abc[3 * k + 1];
-      sa.c = plan->abc[3 * k + 2];
-      if (plan->mode == 0) {
-        sa.lr = hyper->lr;
-        sa.wd = hyper->weight_decay;
-        sa.gamma = hyper->gamma;
-      }
-      sa.wait_limit_ns = limit;
-      const int64_t tiles = sa.total_tiles - sa.tile_begin;
-      cudaError_t e;
+  // arguments of one stage launch (step k, kind) over the tiles of batch bt
+  auto stage_args = [&](int k, int kind, const std::pair<int, int>& bt) {
+    StageArgs sa{};
+    sa.groups = groups;
+    sa.mats = mats;
+    sa.tmaps = ws + plan->off_tmaps;
+    sa.mat_tmaps = ws + plan->off_mat_tmaps;
+    sa.ws = ws;
+    sa.scale = scale;
+    sa.err = err;
+    sa.tile_begin = first_tile(plan, bt.first, kind);
+    sa.total_tiles = first_tile(plan, bt.second, kind);
+    sa.ngroups = static_cast<int32_t>(plan->groups.size());
+    const bool last = k == plan->steps - 1;
+    sa.first = k == 0;
+    // unit-RMS scale: the last Apply keeps O' and its sums of squares; the
+    // update comes after the per-matrix reduction. Diagnostics: the fused
+    // last step records the sums too.
+    sa.last = last && !unit;
+    sa.scale_mode = plan->scale_mode;
+    if ((unit || diag) && last && kind == kApply) {
+      sa.sumsq_per_tile = plan->sumsq_per_tile;
+      sa.sumsq = reinterpret_cast<float*>(ws + plan->off_sumsq);
+    }
+    sa.xsrc = k & 1;
+    sa.a = plan->abc[3 * k];
+    sa.b = plan->abc[3 * k + 1];
+    sa.c = plan->abc[3 * k + 2];
+    if (plan->mode == 0) {
+      sa.lr = hyper->lr;
+      sa.wd = hyper->weight_decay;
+      sa.gamma = hyper->gamma;
+    }
+    sa.wait_limit_ns = limit;
+    sa.chain_sumsq_stage = -1;
+    return sa;
+  };
+  auto launch_one = [&](const StageArgs& sa, int kind, const std::pair<int, int>& bt) -> muon_status_t {
+    const int64_t tiles = sa.total_tiles - sa.tile_begin;
+    cudaError_t e;
+    if (tc) {
+      const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, sms / 2));
+      e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, wide_epilogue(plan, bt, kind, sa.last != 0), stream);
+    } else {
+      const int grid = static_cast<int>(std::min<int64_t>(tiles, 8LL * sms));
+      e = launch_stage_simt(static_cast<StageKind>(kind), sa, grid, stream);
+    }
+    return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+  };
+  if (chained(plan)) {
+    // every stage in one persistent launch (the last Apply too in the
+    // unit-RMS mode), then the last Apply fused with the update
+    const std::pair<int, int> all(0, static_cast<int>(plan->mats.size()));
+    StageArgs sa = stage_args(0, kGram, all);
+    sa.tile_begin = 0;
+    sa.total_tiles = plan->chain_len;
+    sa.chain = reinterpret_cast<const ChainTile*>(ws + plan->off_chain);
+    sa.dep = reinterpret_cast<unsigned*>(ws + plan->off_dep);
+    sa.chain_stages = unit ? 3 * plan->steps : 3 * plan->steps - 1;
+    sa.last = 0;
+    if (unit) {
+      sa.chain_sumsq_stage = 3 * plan->steps - 1;
+      sa.sumsq_per_tile = plan->sumsq_per_tile;
+      sa.sumsq = reinterpret_cast<float*>(ws + plan->off_sumsq);
+    }
+    for (int k = 0; k < 3 * plan->steps; ++k) sa.abc[k] = plan->abc[k];
+    const int pairs = std::max(1, g_chain_pairs[dev]);
+    const int grid = 2 * static_cast<int>(std::min<int64_t>(plan->chain_len, pairs));
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (launch_stage_chain(sa, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    if (!unit) {
+      const StageArgs la = stage_args(plan->steps - 1, kApply, all);
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
-      if (tc) {
-        const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, sms / 2));
-        e = launch_stage_tc(static_cast<StageKind>(kind), sa, grid, wide_epilogue(plan, bt, kind, sa.last != 0), stream);
-      } else {
-        const int grid = static_cast<int>(std::min<int64_t>(tiles, 8LL * sms));
-        e = launch_stage_simt(static_cast<StageKind>(kind), sa, grid, stream);
-      }
-      if (e != cudaSuccess) return MUON_ERR_CUDA;
+      if ((st = launch_one(la, kApply, all)) != MUON_OK) return st;
       if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+    }
+  } else {
+    // one pass of every step per batch: a batch's buffers stay in L2 across its
+    // 3 x steps launches when the batch fits
+    for (const auto& bt : plan->batches)
+    for (int k = 0; k < plan->steps; ++k) {
+      if (first_tile(plan, bt.first, kApply) == first_tile(plan, bt.second, kApply)) break;
+      for (int kind = 0; kind < kNumKinds; ++kind) {
+        const StageArgs sa = stage_args(k, kind, bt);
+        if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+        if ((st = launch_one(sa, kind, bt)) != MUON_OK) return st;
+        if ((st = record(plan, slot++, stream)) != MUON_OK) return st;
+      }
     }
   }
   if (unit || diag) {
@@ -833,6 +961,16 @@ muon_status_t muon_plan_set_diagnostics(muon_plan_t plan, float* out) {
   plan->diag = out;
   make_launch_list(plan);
   plan->events.clear();  // the launch list may have changed: timing must be set again
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_chaining(muon_plan_t plan, int on, int window) {
+  if (!plan || window < 0) return MUON_ERR_INVALID_ARG;
+  plan->chain_on = on != 0;
+  plan->chain_window = window;
+  make_launch_list(plan);
+  plan->events.clear();    // the launch list may have changed: timing must be set again
+  plan->uploaded_ws = nullptr;  // the tile list is rebuilt by the next execute
   return MUON_OK;
 }
 
@@ -920,6 +1058,18 @@ void muon_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns < 1000 ? 1000 : ns, std::memory_order_relaxed);
 }
 
+muon_status_t muon_dep_wait_probe(const uint32_t* counter, uint32_t target, uint64_t limit_ns,
+                                  void* stream) {
+  if (!counter) return MUON_ERR_INVALID_ARG;
+  int dev = 0;
+  muon_status_t st = device_setup(&dev);
+  if (st != MUON_OK) return st;
+  return launch_dep_wait_probe(counter, target, g_err_ptr[dev], limit_ns,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MUON_OK
+             : MUON_ERR_CUDA;
+}
+
 muon_status_t muon_wait_probe(const int* flag, uint64_t limit_ns, void* stream) {
   if (!flag) return MUON_ERR_INVALID_ARG;
   int dev = 0;
@@ -997,6 +1147,21 @@ cudaError_t launch_blob_copy(void* dst, const void* src, size_t bytes, cudaStrea
 cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limit_ns,
                               cudaStream_t stream) {
   wait_probe_kernel<<<1, 1, 0, stream>>>(flag, err, limit_ns);
+  return cudaGetLastError();
+}
+
+namespace {
+// The chained launch's dependency wait, alone: on expiry, the timeout bit.
+__global__ void dep_wait_probe_kernel(const unsigned* counter, unsigned target, int* err,
+                                      unsigned long long limit_ns) {
+  volatile int no_abort = 0;
+  if (!ptx::dep_wait(counter, target, err, limit_ns, &no_abort)) atomicOr(err, kErrTimeout);
+}
+}  // namespace
+
+cudaError_t launch_dep_wait_probe(const uint32_t* counter, uint32_t target, int* err,
+                                  unsigned long long limit_ns, cudaStream_t stream) {
+  dep_wait_probe_kernel<<<1, 1, 0, stream>>>(counter, target, err, limit_ns);
   return cudaGetLastError();
 }
 

@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(kEwThreads, kEwMinBlocks) ew_kernel(const __gr
     a.scale[mi] = static_cast<float>(1.0 / (sqrt(s) + static_cast<double>(a.eps)));
     if (a.diag) a.diag[2 * md.caller] = static_cast<float>(sqrt(s));
     a.counter[mi] = 0u;
+    if (a.dep) a.dep[mi] = 0u;  // the chained stage launch that follows counts from zero
   }
 }
 

@@ -19,6 +19,14 @@ cudaError_t launch_elementwise(const EwArgs& args, cudaStream_t stream);
 cudaError_t launch_stage_tc(StageKind kind, const StageArgs& args, int grid, bool wide,
                             cudaStream_t stream);
 
+// Every Gram, Poly and Apply stage listed in args.chain (tiles
+// [tile_begin, total_tiles)) in one persistent launch, with per-matrix
+// dependency counters args.dep (reset to zero by the elementwise kernel).
+// The grid must not exceed 2 * chain_max_pairs(): every CTA pair must be
+// resident at once.
+cudaError_t launch_stage_chain(const StageArgs& args, int grid, cudaStream_t stream);
+cudaError_t chain_max_pairs(int* pairs);
+
 // Every Newton-Schulz step and the update for the small matrices, one CTA
 // per matrix (bf16 precision).
 cudaError_t launch_small(const SmallArgs& args, int grid, cudaStream_t stream);
@@ -53,5 +61,10 @@ cudaError_t launch_blob_copy(void* dst, const void* src, size_t bytes, cudaStrea
 // the timeout path. Sets the timeout bit of `err` when the limit passes.
 cudaError_t launch_wait_probe(const int* flag, int* err, unsigned long long limit_ns,
                               cudaStream_t stream);
+
+// The chained launch's dependency wait on `counter` >= target, alone, for
+// the tests of its timeout path.
+cudaError_t launch_dep_wait_probe(const uint32_t* counter, uint32_t target, int* err,
+                                  unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace muon

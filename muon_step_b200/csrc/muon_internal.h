@@ -100,6 +100,19 @@ struct MatDesc {
   int64_t ew_tiles;      // number of elementwise tiles
 };
 
+// One tile of the chained launch's list: stage = 3 * step + kind (Gram 0,
+// Poly 1, Apply 2), tile = index within the matrix's table of that kind.
+struct ChainTile {
+  int32_t mat;    // internal matrix index
+  int32_t stage;
+  int32_t tile;
+  int32_t pad;
+};
+
+// Epilogue warps per tile of the chained launch (8 per CTA, two CTAs): each
+// adds one to its matrix's dependency counter when its stores have landed.
+constexpr int kChainArrivals = 16;
+
 // Per-launch arguments of the Newton-Schulz stage kernels.
 struct StageArgs {
   const GroupDesc* groups;
@@ -121,6 +134,13 @@ struct StageArgs {
   int32_t sumsq_per_tile; // > 0: the last step records sums of squares of X' (per tile slots)
   float* sumsq;           // ... into sumsq[tile * sumsq_per_tile + slot]
   uint64_t wait_limit_ns; // bound on every spin-wait
+  // chained launch: every Gram / Poly / Apply stage of the schedule in one
+  // persistent kernel, tiles taken in the order of a host-built list
+  const ChainTile* chain; // [total_tiles]
+  unsigned* dep;          // per matrix: epilogue-warp tile completions so far this execute
+  int32_t chain_sumsq_stage;  // stage whose Apply records sums of squares (-1: none)
+  int32_t chain_stages;       // tiles of later stages in the list are skipped
+  float abc[kMaxSteps * 3];   // every step's coefficients
 };
 
 // Elementwise-stage arguments (momentum + Nesterov + Frobenius partials + cast).
@@ -140,6 +160,7 @@ struct EwArgs {
   int32_t split;          // bf16 mode: the iterate as bf16 high + low parts (else fp32)
   float mu, eps;
   float* diag;            // optional: diag[2 caller] = ||N||_F
+  unsigned* dep;          // optional: chained-launch dependency counters, reset per matrix
 };
 
 // Small-matrix kernel arguments (one CTA per matrix, every step on chip).

@@ -298,3 +298,52 @@ __device__ __forceinline__ void umma_commit_pair_self(uint64_t* bar) {
 
 }  // namespace ptx
 }  // namespace muon
+
+namespace muon {
+namespace ptx {
+
+// ---------------------------------------------------------------- cross-CTA dependencies
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's completed async-proxy (TMA) global writes before its
+// later generic accesses, and its generic acquires before later async-proxy
+// (TMA) global reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *ctr >= target (acquire), then order later TMA reads after it.
+// Returns false when the time limit passes, another role of the CTA has
+// raised `abort_flag`, or another CTA has set the timeout bit in `err`.
+__device__ __forceinline__ bool dep_wait(const unsigned* ctr, uint32_t target, const int* err,
+                                         uint64_t limit_ns, volatile int* abort_flag) {
+  if (ld_acquire_gpu(ctr) >= target) {
+    fence_proxy_async_global();
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  for (uint64_t it = 0; it < kSpinBackstop; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(ctr) >= target) {
+      fence_proxy_async_global();
+      return true;
+    }
+    if (*abort_flag) return false;
+    if ((it & 15) == 0) {
+      if (*reinterpret_cast<const volatile int*>(err) & 1) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+  return false;
+}
+
+}  // namespace ptx
+}  // namespace muon

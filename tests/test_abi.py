@@ -156,6 +156,16 @@ def expected_workspace(shapes, prec):
         slots = 1
     off = al(off + apply_tiles * slots * 4, 256)
     off = al(off + nm * 4, 256)
+    # chained launch (bf16): a 16-byte entry per tile of every stage of every
+    # step of every grouped matrix, then a dependency counter per matrix
+    if prec == MUON_NS_BF16:
+        chain = 0
+        for (r, c), mem in groups.items():
+            if r * c > TINY and (r > 128 or c > 512):
+                pb = math.ceil(r / 256)
+                chain += len(mem) * 10 * (2 * (pb * (pb + 1) // 2) + pb * math.ceil(c / 256))
+        off = al(off + chain * 16, 256)
+        off = al(off + nm * 4, 256)
     off = al(off, 1024)
     for (r, c), mem in sorted(groups.items(), key=lambda kv: order.index(kv[0])):
         k = len(mem)
@@ -197,7 +207,9 @@ def launch_list(lib, shapes, prec=MUON_NS_BF16):
 
 
 def test_launch_list(lib):
-    grouped = [1, 2, 3] * 9 + [1, 2, 4]
+    # bf16: every stage in one chained launch (10), then the last Apply with the update (4)
+    grouped = [10, 4]
+    stagewise = [1, 2, 3] * 9 + [1, 2, 4]
     # matrices of at most 4096 elements run with fp32 operands in the tiny-matrix kernel (kind 9)
     assert launch_list(lib, [(64, 64)]) == [0, 9]
     assert launch_list(lib, [(1, 1), (7, 100), (1, 4096), (4096, 1), (32, 128)]) == [0, 9]
@@ -213,9 +225,28 @@ def test_launch_list(lib):
     assert launch_list(lib, [(129, 129)]) == [0] + grouped
     assert launch_list(lib, [(64, 64), (300, 400)]) == [0, 9] + grouped
     assert launch_list(lib, [(65, 65), (100, 300), (300, 400)]) == [0, 5, 8] + grouped
-    # the fp32 validation precision runs every matrix on the grouped fp32 kernels
-    assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + grouped
-    assert launch_list(lib, [(2, 3)], MUON_NS_FP32) == [0] + grouped
+    # the fp32 validation precision runs every matrix on the grouped fp32 kernels, stage by stage
+    assert launch_list(lib, [(64, 64)], MUON_NS_FP32) == [0] + stagewise
+    assert launch_list(lib, [(2, 3)], MUON_NS_FP32) == [0] + stagewise
+    assert launch_list(lib, [(300, 400)], MUON_NS_FP32) == [0] + stagewise
+
+
+def test_chaining_can_be_turned_off(lib):
+    st, plan = create(lib, [(300, 400), (64, 64)])
+    cnt = ctypes.c_int()
+    kinds = (ctypes.c_int * 128)()
+
+    def kinds_now():
+        assert lib.muon_plan_launches(plan, ctypes.byref(cnt), kinds, 128) == MUON_OK
+        return list(kinds[:cnt.value])
+
+    assert kinds_now() == [0, 9, 10, 4]
+    assert lib.muon_plan_set_chaining(plan, 0, 0) == MUON_OK
+    assert kinds_now() == [0, 9] + [1, 2, 3] * 9 + [1, 2, 4]
+    assert lib.muon_plan_set_chaining(plan, 1, 7) == MUON_OK
+    assert kinds_now() == [0, 9, 10, 4]
+    assert lib.muon_plan_set_chaining(plan, 1, -1) == MUON_ERR_INVALID_ARG
+    lib.muon_plan_destroy(plan)
 
 
 def test_scale_modes_change_the_launch_list(lib):
@@ -228,10 +259,11 @@ def test_scale_modes_change_the_launch_list(lib):
         return list(kinds[:cnt.value])
 
     shape = kinds_now()
-    assert shape[-1] == 4
-    # unit-RMS: the last Apply keeps O', then a per-matrix reduction and an update pass
+    assert shape[-2:] == [10, 4]
+    # unit-RMS: the chained launch keeps O' from the last Apply, then a
+    # per-matrix reduction and an update pass
     assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
-    assert kinds_now() == shape[:-1] + [3, 6, 7]
+    assert kinds_now() == shape[:-1] + [6, 7]
     assert lib.muon_plan_set_scale_mode(plan, 2) == MUON_OK
     assert kinds_now() == shape
     assert lib.muon_plan_set_scale_mode(plan, 3) == MUON_ERR_INVALID_ARG
@@ -247,7 +279,7 @@ def test_scale_modes_change_the_launch_list(lib):
     assert lib.muon_plan_set_diagnostics(plan, ctypes.c_void_p(FAKE)) == MUON_OK
     assert kinds_now() == shape + [6]
     assert lib.muon_plan_set_scale_mode(plan, 1) == MUON_OK
-    assert kinds_now() == shape[:-1] + [3, 6, 7]
+    assert kinds_now() == shape[:-1] + [6, 7]
     assert lib.muon_plan_set_diagnostics(plan, None) == MUON_OK
     assert lib.muon_plan_set_scale_mode(plan, 0) == MUON_OK
     assert kinds_now() == shape
@@ -291,6 +323,12 @@ def test_ns_plan_arguments(lib):
 def test_timing_events_need_two_per_launch(lib):
     st, plan = create(lib, [(300, 300)])
     ev = (ctypes.c_void_p * 62)(*([FAKE] * 62))
+    # chained: the elementwise launch, the chain and the fused last Apply
+    assert lib.muon_plan_set_events(plan, ev, 5) == MUON_ERR_INVALID_ARG
+    assert lib.muon_plan_set_events(plan, ev, 6) == MUON_OK
+    assert lib.muon_plan_set_events(plan, None, 0) == MUON_OK
+    # stage by stage: 1 + 30 launches
+    assert lib.muon_plan_set_chaining(plan, 0, 0) == MUON_OK
     assert lib.muon_plan_set_events(plan, ev, 61) == MUON_ERR_INVALID_ARG
     assert lib.muon_plan_set_events(plan, ev, 62) == MUON_OK
     assert lib.muon_plan_set_events(plan, None, 0) == MUON_OK
@@ -334,7 +372,7 @@ def test_l2_batching_repeats_the_stage_launches_per_batch(lib):
         return list(kinds[:cnt.value])
 
     one_pass = [1, 2, 3] * 9 + [1, 2, 4]
-    assert kinds_now() == [0, 5] + one_pass
+    assert kinds_now() == [0, 5, 10, 4]  # chained by default; L2 batching runs stage by stage
     ws0 = ctypes.c_size_t()
     assert lib.muon_plan_workspace_size(plan, ctypes.byref(ws0)) == MUON_OK
     # one 300 x 400 matrix needs 6*300*400 + 4*300*304 = 1,084,800 bytes of buffers
@@ -348,7 +386,7 @@ def test_l2_batching_repeats_the_stage_launches_per_batch(lib):
     assert lib.muon_plan_workspace_size(plan, ctypes.byref(ws1)) == MUON_OK
     assert ws1.value == ws0.value
     assert lib.muon_plan_set_l2_batching(plan, 0) == MUON_OK
-    assert kinds_now() == [0, 5] + one_pass
+    assert kinds_now() == [0, 5, 10, 4]
     lib.muon_plan_destroy(plan)
 
 
@@ -382,7 +420,7 @@ if given is not None:
                     for a, b in shapes)
         want = [0] + ([5] if small else []) + ([8] if mid else []) + ([9] if tiny else [])
         if large:
-            want += [1, 2, 3] * 9 + [1, 2, 4]
+            want += [10, 4] if tc else [1, 2, 3] * 9 + [1, 2, 4]
         assert launch_list(lib, shapes, prec) == want
 
 

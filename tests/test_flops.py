@@ -73,7 +73,7 @@ def test_one_cta_kinds_follow_the_planner():
         _, kinds = _plan_flops([shape], 0)
         want = bench.one_cta_kind(*shape)
         if want is None:
-            assert kinds >= {1, 2, 3, 4} and not kinds & {5, 8, 9}, shape
+            assert kinds == {0, 10, 4} and not kinds & {5, 8, 9}, shape
         else:
             assert kinds == {0, want}, shape
         _, kinds32 = _plan_flops([shape], 1)

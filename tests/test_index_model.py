@@ -346,3 +346,130 @@ def tiny_kernel_accesses(n, m):
 def test_tiny_kernel_stays_inside_its_buffers(n, m):
     assert n * m <= TINY_MAX
     tiny_kernel_accesses(n, m)
+
+
+# ---------------------------------------------------------------- chained launch
+
+CHAIN_ARRIVALS = 16  # epilogue warps per tile (8 per CTA, two CTAs)
+
+
+def build_chain(shapes, npairs, steps=10, window=0):
+    """The planner's tile list of the chained launch: a window of matrices in
+    flight, in rounds; each round lists the next stage of every matrix in the
+    window (all its tiles); finished matrices leave for the next ones."""
+    groups = groups_of(shapes)
+    per, _, _ = tile_tables(groups)
+    mats = []  # (group, index in group)
+    for g, (r, c, count, _) in enumerate(groups):
+        mats += [(g, b) for b in range(count)]
+    grouped = [k for k, (g, b) in enumerate(mats) if sum(per[g]) > 0]
+    if not grouped:
+        return groups, per, mats, []
+    if window <= 0:
+        mean = sum(sum(per[mats[k][0]]) / 3.0 for k in grouped) / len(grouped)
+        window = math.ceil(2.0 * max(npairs, 1) / max(mean, 1.0))
+    window = max(1, min(window, len(grouped)))
+    out, act, nxt = [], [], 0
+    while nxt < len(grouped) or act:
+        while len(act) < window and nxt < len(grouped):
+            act.append([grouped[nxt], 0])
+            nxt += 1
+        for x in act:
+            g = mats[x[0]][0]
+            out += [(x[0], x[1], u) for u in range(per[g][x[1] % 3])]
+            x[1] += 1
+        act = [x for x in act if x[1] < 3 * steps]
+    return groups, per, mats, out
+
+
+def chain_need(per_g, stage):
+    """Counter value at which every tile of the matrix's earlier stages has
+    finished (the kernel's chain_pos)."""
+    g0, p0, a0 = per_g
+    step, kind = divmod(stage, 3)
+    return CHAIN_ARRIVALS * (step * (g0 + p0 + a0) + (g0 if kind >= 1 else 0) + (p0 if kind >= 2 else 0))
+
+
+def simulate_chain(shapes, npairs, steps=10, window=0, chain_stages=None):
+    """Every pair takes its tiles (t = pair, pair + npairs, ...) in list order;
+    a tile starts when its matrix's counter has reached its target and adds
+    CHAIN_ARRIVALS when it finishes (its time: its K blocks). Returns the
+    makespan; fails on a deadlock."""
+    groups, per, mats, tiles = build_chain(shapes, npairs, steps, window)
+    nst = 3 * steps if chain_stages is None else chain_stages
+    dep = [0] * len(mats)
+    pos = [p for p in range(npairs)]        # next list index of each pair
+    busy = [0.0] * npairs                   # time each pair becomes free
+    now, done, running = 0.0, 0, []         # running: (finish time, pair, matrix)
+    todo = sum(1 for _, s, _ in tiles if s < nst)
+    import heapq
+    while done < todo:
+        progressed = False
+        for p in range(npairs):
+            if busy[p] > now:
+                continue
+            while pos[p] < len(tiles) and tiles[pos[p]][1] >= nst:
+                pos[p] += npairs            # skipped by every role
+            if pos[p] >= len(tiles):
+                continue
+            mat, stage, u = tiles[pos[p]]
+            g = mats[mat][0]
+            if dep[mat] < chain_need(per[g], stage):
+                continue
+            r, c, _, _ = groups[g]
+            k = c if stage % 3 == 0 else r
+            t_end = now + cdiv(k, BK)
+            heapq.heappush(running, (t_end, p, mat))
+            busy[p] = t_end
+            pos[p] += npairs
+            progressed = True
+        if running:
+            t_end, p, mat = heapq.heappop(running)
+            now = max(now, t_end)
+            dep[mat] += CHAIN_ARRIVALS
+            done += 1
+        elif not progressed:
+            raise AssertionError("deadlock: no pair can start a tile")
+    return now, dep, per, mats, tiles
+
+
+@pytest.mark.parametrize("shapes,npairs", [
+    ([(1024, 1024)] * 64, 74),
+    ([(512, 512)] * 40 + [(512, 2048)] * 7, 74),
+    ([(4096, 4096)] * 4 + [(4096, 14336)] * 2 + [(14336, 4096)], 74),
+    ([(300, 520), (520, 300), (257, 129), (1000, 300), (600, 600)], 3),
+    ([(1024, 1024)] * 5, 1),
+])
+def test_chain_list_covers_every_stage_once_and_never_deadlocks(shapes, npairs):
+    for window in (0, 1, 3):
+        for stages in (None, 29):
+            _, dep, per, mats, tiles = simulate_chain(shapes, npairs, window=window, chain_stages=stages)
+            # every tile of every stage of every grouped matrix, once
+            seen = {}
+            for mat, stage, u in tiles:
+                seen[(mat, stage, u)] = seen.get((mat, stage, u), 0) + 1
+            assert all(v == 1 for v in seen.values())
+            for k, (g, _) in enumerate(mats):
+                if sum(per[g]) == 0:
+                    continue
+                for stage in range(30):
+                    assert all((k, stage, u) in seen for u in range(per[g][stage % 3]))
+                # the counter ends at the arrivals of every tile that ran
+                nst = 30 if stages is None else stages
+                assert dep[k] == chain_need(per[g], nst), (k, dep[k])
+            # a tile's target is reached only by tiles listed before it
+            first_pos = {}
+            for i, (mat, stage, u) in enumerate(tiles):
+                first_pos.setdefault((mat, stage), i)
+            for i, (mat, stage, u) in enumerate(tiles):
+                if stage > 0:
+                    assert first_pos[(mat, stage - 1)] < first_pos[(mat, stage)] <= i
+
+
+def test_chain_targets_are_prefix_sums_of_earlier_stages():
+    per_g = (10, 10, 16)
+    assert chain_need(per_g, 0) == 0
+    assert chain_need(per_g, 1) == 16 * 10
+    assert chain_need(per_g, 2) == 16 * 20
+    assert chain_need(per_g, 3) == 16 * 36
+    assert chain_need(per_g, 29) == 16 * (9 * 36 + 20)

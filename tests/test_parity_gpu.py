@@ -447,3 +447,74 @@ def test_copy_segments_moves_every_segment():
     assert lib.muon_copy_segments(segs, len(cuts), ws.data_ptr(), ws.numel(), stream) == 0
     torch.cuda.synchronize()
     assert torch.equal(dst, want)
+
+
+def test_dependency_wait_timeout_is_reported_and_the_context_survives():
+    """The chained launch's dependency wait, on a counter nothing advances,
+    gives up after its limit and reports MUON_ERR_TIMEOUT; the same wait on a
+    counter that has reached its target passes; the library still runs."""
+    import muon_step_b200 as ms
+    counter = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ms.dep_wait_probe(counter, 16, 2_000_000)  # 2 ms, the signal is withheld
+    assert ms.sync_status() == 5                # MUON_ERR_TIMEOUT
+    assert ms.sync_status() == 0
+    counter.fill_(16)
+    ms.dep_wait_probe(counter, 16, 2_000_000)
+    assert ms.sync_status() == 0
+    wl = workloads.make_random([(300, 520)], device="cuda", seed=2)
+    assert check_step(wl, "bf16")["O_over_tol"] <= 1.0
+
+
+CHAIN_SHAPES = [(300, 520), (520, 300), (257, 129), (1000, 300), (600, 600), (1024, 1024),
+                (64, 64), (100, 120), (300, 520)]
+
+
+@pytest.mark.parametrize("scale_mode", ["shape", "unit_rms", "none"])
+@pytest.mark.parametrize("window", [0, 1, 50])
+def test_chained_launch_is_bit_identical_to_stagewise(scale_mode, window):
+    """Every Newton-Schulz stage in one chained launch (per-matrix dependency
+    counters, a window of matrices in flight) gives the same bits as one
+    launch per stage: W, M, O' and the diagnostics, over two steps."""
+    import muon_step_b200 as ms
+
+    a = workloads.make_random(CHAIN_SHAPES, device="cuda", seed=79)
+    b = workloads.make_random(CHAIN_SHAPES, device="cuda", seed=79)
+    Oa = [torch.empty_like(w) for w in a.W]
+    Ob = [torch.empty_like(w) for w in b.W]
+    pa = ms.MuonPlan([(a.W[k], a.G[k], a.M[k], Oa[k]) for k in range(a.count)], scale_mode=scale_mode)
+    pb = ms.MuonPlan([(b.W[k], b.G[k], b.M[k], Ob[k]) for k in range(b.count)], scale_mode=scale_mode)
+    pa.set_chaining(True, window)
+    pb.set_chaining(False)
+    da = torch.zeros((a.count, 2), device="cuda")
+    db = torch.zeros((b.count, 2), device="cuda")
+    pa.set_diagnostics(da)
+    pb.set_diagnostics(db)
+    assert 10 in pa.launches() and 10 not in pb.launches()
+    for _ in range(2):
+        pa.execute()
+        pb.execute()
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for k in range(a.count):
+        assert torch.equal(a.W[k], b.W[k]), k
+        assert torch.equal(a.M[k], b.M[k]), k
+        assert torch.equal(Oa[k], Ob[k]), k
+    assert torch.equal(da, db)
+
+
+def test_chained_orthogonalize_matches_stagewise():
+    import muon_step_b200 as ms
+
+    rng = torch.Generator(device="cuda").manual_seed(83)
+    xs = [torch.randn(n, m, generator=rng, device="cuda") for n, m in CHAIN_SHAPES]
+    outs = []
+    for chain in (True, False):
+        o = [torch.empty_like(x) for x in xs]
+        plan = ms.NsPlan(list(zip(xs, o)))
+        plan.set_chaining(chain)
+        plan.execute()
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert ms.sync_status() == 0
+    for oa, ob in zip(*outs):
+        assert torch.equal(oa, ob)
