@@ -70,8 +70,9 @@ def parse_args():
     ap.add_argument("--cpu-sample", type=int, default=6, help="matrices in the CPU-baseline sample")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
     ap.add_argument("--count", type=int, default=None,
-                    help="sweep workloads only: this many matrices instead of ~16 GB of state "
-                         "(small cases for profiling; not a benchmark line)")
+                    help="a smaller case of the workload for profiling (not a benchmark line): "
+                         "this many layers (dense_d4096), experts (moe_64x3) or matrices (the "
+                         "others)")
     return ap.parse_args()
 
 
@@ -520,6 +521,19 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def count_kwargs(config, count):
+    """Keyword that shrinks a workload to `count` units (None: full size)."""
+    if count is None:
+        return {}
+    if config == "dense_d4096":
+        return {"layers": count}
+    if config == "moe_64x3":
+        return {"experts": count}
+    if config == "single_256x512":
+        raise SystemExit("single_256x512 has one matrix")
+    return {"count": count}
+
+
 def _small_kwargs(config):
     # the reference arm needs only one matrix of the workload's shape
     if config == "batch64_1024":
@@ -657,10 +671,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    if args.count is not None and not args.config.startswith("sweep_"):
-        raise SystemExit("--count applies to the sweep workloads only")
-    wl = workloads.make(args.config, device=dev,
-                        **({"count": args.count} if args.count is not None else {}))
+    wl = workloads.make(args.config, device=dev, **count_kwargs(args.config, args.count))
     h = wl.hyper
     params = [(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)]
     plan = ms.MuonPlan(params, precision=args.precision)

@@ -99,7 +99,7 @@ constexpr int kTmapBytes = 128;
 
 // Facts of a tile kind that do not depend on the launch layout. Slot use:
 //   Gram       [bf16 out | bf16 mirror out]                            4 KB
-//   Poly       [bf16 A in | bf16 out | bf16 mirror out]                6 KB
+//   Poly       [bf16 A in, then mirror out | bf16 out]                 4 KB
 //   Apply      [bf16 iterate high in / out | bf16 low in / out]        4 KB
 //   ApplyLast  [bf16 high in | bf16 low in, then fp32 O out | fp32 W in / out]  8 KB
 template <int KIND>
@@ -107,12 +107,11 @@ struct KindT {
   static constexpr bool kApplyLike = (KIND == kApply || KIND == kApplyLast);
   static constexpr int kTiles = kApplyLike ? kApply : KIND;  // which tile tables to walk
   static constexpr bool kInput = (KIND != kGram);            // the epilogue loads inputs
-  static constexpr int kSlotUse = (KIND == kApplyLast) ? 2 * kEpiF32
-                                  : (KIND == kPoly)    ? 3 * kEpiB16
-                                                       : 2 * kEpiB16;
+  static constexpr int kSlotUse = (KIND == kApplyLast) ? 2 * kEpiF32 : 2 * kEpiB16;
   // symmetric kinds: where the direct and mirrored outputs sit in a slot
+  // (Poly's mirror takes the area of its A input once every lane has read it)
   static constexpr int kOffSymOut = (KIND == kPoly) ? kEpiB16 : 0;
-  static constexpr int kOffSymMirror = kOffSymOut + kEpiB16;
+  static constexpr int kOffSymMirror = (KIND == kPoly) ? 0 : kEpiB16;
 };
 
 // Launch layout: ring depth, epilogue warps (one per TMEM lane quarter, or
@@ -137,17 +136,16 @@ struct Layout {
 template <int KIND, bool WIDE>
 struct StageLayout {
   static constexpr bool kWide = WIDE || KIND == kApply;
-  static constexpr int kStages = (KIND == kGram)   ? (kWide ? 5 : 6)
-                                 : (KIND == kPoly) ? (kWide ? 4 : 5)
-                                 : (KIND == kApply) ? 5
-                                                    : (kWide ? 3 : 4);
+  static constexpr int kStages = (KIND == kGram || KIND == kPoly) ? (kWide ? 5 : 6)
+                                 : (KIND == kApply)                ? 5
+                                                                   : (kWide ? 3 : 4);
   static constexpr int kEpiSlots = (KIND == kApplyLast && !kWide) ? 3 : 2;
   using L = Layout<kStages, kWide ? 8 : 4, KindT<KIND>::kSlotUse, kEpiSlots>;
 };
 
 // The chained launch runs Gram, Poly and Apply tiles with one layout: eight
-// epilogue warps, slots sized for Poly, four ring stages.
-using ChainL = Layout<4, 8, 3 * kEpiB16, 2>;
+// epilogue warps, two 4 KB slots each, five ring stages.
+using ChainL = Layout<5, 8, 2 * kEpiB16, 2>;
 static_assert(ChainL::kSmem <= 227 * 1024, "shared memory budget");
 
 constexpr int kOffLow = kEpiB16;   // low part of the iterate in Apply-like slots
@@ -359,7 +357,9 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p
     *reinterpret_cast<Bf16x8*>(st_direct + sw64_chunk(lane, q)) = pk;
   }
   if (mirror) {
-    // transposed chunk: row e of the mirror holds column e of this chunk
+    // transposed chunk: row e of the mirror holds column e of this chunk (for
+    // Poly in the A input's area: every lane has read its row of A first)
+    if (KIND == kPoly) __syncwarp();
     __nv_bfloat16* m16 = reinterpret_cast<__nv_bfloat16*>(st_mirror);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -638,16 +638,43 @@ struct EpiState {
   uint32_t eload_phase = 0;  // bit i: phase of slot i's load barrier
 };
 
+// The last Apply's epilogue inputs that the MMA does not bring into L2 (the
+// iterate's low part and the caller's W) for this warp's chunks of tile
+// `tc`: L2 prefetches, issued one tile ahead, so that the epilogue's loads
+// of them wait on L2 rather than DRAM.
+template <typename L>
+__device__ __forceinline__ void prefetch_last_inputs(const StageArgs& a, const TileCoord& tc,
+                                                     uint32_t rank, int ew, int warp) {
+  const GroupDesc& gd = a.groups[tc.g];
+  const int row0 = tc.I * kPairTile + static_cast<int>(rank) * kHalf + (warp & 3) * 32;
+  if (row0 >= gd.r) return;
+  const int bz = static_cast<int>(tc.b);
+  const int mat = gd.first_mat + bz;
+  const MatDesc& md = a.mats[mat];
+  const bool w_tma = md.W && last_by_tma(md);
+  const int ch_begin = (ew / 4) * L::kChunksPerWarp;
+  for (int ch = ch_begin; ch < ch_begin + L::kChunksPerWarp; ++ch) {
+    const int col0 = tc.J * kPairTile + ch * 32;
+    if (col0 >= gd.c) break;
+    ptx::tma_prefetch_3d(tmap(a, tc.g, kTmXloE), col0, row0, bz);
+    if (w_tma)
+      ptx::tma_prefetch_3d(mat_tmap(a, mat, kMtW), md.transposed ? row0 : col0,
+                           md.transposed ? col0 : row0, 0);
+  }
+}
+
 // Epilogue warp: one tile. With `dep` set (chained launch) the warp first
 // waits until the tile's inputs have landed (counter >= need) and, once its
-// own stores have landed, adds one to the matrix's counter. Returns false
-// when a wait gives up (the pair has been aborted).
+// own stores have landed, adds one to the matrix's counter. `next` (the last
+// Apply) is the pair's next tile, whose inputs are prefetched into L2.
+// Returns false when a wait gives up (the pair has been aborted).
 template <int KIND, typename L>
 __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p, const Smem& s,
                                               const TileCoord& tc, int64_t t_apply, uint32_t rank,
                                               int ew, int warp, int lane, uint32_t tmem_base,
                                               EpiState& es, const uint32_t* leader_tempty,
-                                              uint64_t limit, unsigned* dep, uint32_t need) {
+                                              uint64_t limit, unsigned* dep, uint32_t need,
+                                              const TileCoord* next = nullptr) {
   using K = KindT<KIND>;
   const int quarter = warp & 3;  // TMEM lanes this warp may read: 32 * quarter ...
   const int ch_begin = (ew / 4) * L::kChunksPerWarp;  // this warp's share of the columns
@@ -710,6 +737,7 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
       ptx::bulk_wait_read<0>();  // the previous tile's stores have read every slot
       for (int ch = ch_begin; ch < ch_begin + D; ++ch)
         if (live_chunk(ch)) issue_load(ch);
+      if (KIND == kApplyLast && next != nullptr) prefetch_last_inputs<L>(a, *next, rank, ew, warp);
     }
   }
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -901,8 +929,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(StageLayout<KIND, WI
     bool ok = true;
     for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
+      const bool has_next = KIND == kApplyLast && t + npairs < a.total_tiles;
+      const TileCoord nx = has_next ? decode_tile<KIND>(a, t + npairs) : tc;
       ok = epilogue_tile<KIND, L>(a, p, s, tc, t, rank, ew, warp, lane, tmem_base, es, leader_tempty,
-                                  limit, nullptr, 0u);
+                                  limit, nullptr, 0u, has_next ? &nx : nullptr);
     }
     if (lane == 0) ptx::bulk_wait<0>();
     if (!ok) linger();
