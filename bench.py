@@ -841,7 +841,7 @@ def main():
         ks = list(range(min(args.cpu_sample, wl.count)))
         mats = [(wl.W[k].double().cpu().numpy(), wl.G[k].double().cpu().numpy(),
                  wl.M[k].double().cpu().numpy()) for k in ks]
-        rate, dt, done = cpu_oracle_rate(mats, h, budget_s=30.0)
+        rate, dt, done = cpu_oracle_rate(mats, h, budget_s=20.0)
         cpu = {"value": rate, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                "sample": f"{done} of {wl.count} matrices of {args.config}, {dt:.1f} s of float64 numpy"}
 

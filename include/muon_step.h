@@ -176,7 +176,11 @@ MUON_API muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes)
  * list keeps `window` matrices in flight at a time (0: chosen from the tile
  * counts), so their buffers can stay in L2 from one stage to the next.
  * on = 0: one launch per stage and step. Both give bit-identical results.
- * Timing events must be set again afterwards. */
+ * The chained launch sizes its grid so that all its CTA pairs are resident
+ * at once on an otherwise idle GPU; work of other streams that occupies SMs
+ * when it starts can hold some pairs back, and the bounded waits then report
+ * MUON_ERR_TIMEOUT (use on = 0 in that setting). Timing events must be set
+ * again afterwards. */
 MUON_API muon_status_t muon_plan_set_chaining(muon_plan_t plan, int on, int window);
 
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */

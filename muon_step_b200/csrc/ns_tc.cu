@@ -327,13 +327,16 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p
                                               uint8_t* slot, const float (&v)[32], int lane) {
   float out[32];
   if (KIND == kGram) {
-    float s2 = 1.f;
+    // step one folds s^2; later steps store the product as it is (s^2 = 1)
     if (p.first) {
-      const float s = a.scale[gd.first_mat + tc.b];
-      s2 = s * s;
-    }
+      const float sc = a.scale[gd.first_mat + tc.b];
+      const float s2 = sc * sc;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) out[e] = s2 * v[e];
+      for (int e = 0; e < 32; ++e) out[e] = s2 * v[e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) out[e] = v[e];
+    }
   } else {
     // the A chunk, bf16 with 64-byte swizzle, in the slot's input area
 #pragma unroll
@@ -377,7 +380,8 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p
 }
 
 // X' (or O') = alpha (a X + acc) for one warp's 32 x 32 chunk; X = high +
-// low parts from the slot's two bf16 input areas.
+// low parts from the slot's two bf16 input areas. alpha is the step-one
+// scale s, and 1 on later steps (no multiply then: the same values).
 __device__ __forceinline__ void apply_values(const StepP& p, float alpha, const uint8_t* slot,
                                              const float (&v)[32], int lane, float (&x)[32]) {
 #pragma unroll
@@ -389,9 +393,13 @@ __device__ __forceinline__ void apply_values(const StepP& p, float alpha, const 
       const float2 fh = __bfloat1622float2(h.v[k]);
       const float2 fl = __bfloat1622float2(l.v[k]);
       const int e = 8 * q + 2 * k;
-      x[e] = alpha * fmaf(p.a, fh.x + fl.x, v[e]);
-      x[e + 1] = alpha * fmaf(p.a, fh.y + fl.y, v[e + 1]);
+      x[e] = fmaf(p.a, fh.x + fl.x, v[e]);
+      x[e + 1] = fmaf(p.a, fh.y + fl.y, v[e + 1]);
     }
+  }
+  if (p.first) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = alpha * x[e];
   }
 }
 
@@ -638,43 +646,16 @@ struct EpiState {
   uint32_t eload_phase = 0;  // bit i: phase of slot i's load barrier
 };
 
-// The last Apply's epilogue inputs that the MMA does not bring into L2 (the
-// iterate's low part and the caller's W) for this warp's chunks of tile
-// `tc`: L2 prefetches, issued one tile ahead, so that the epilogue's loads
-// of them wait on L2 rather than DRAM.
-template <typename L>
-__device__ __forceinline__ void prefetch_last_inputs(const StageArgs& a, const TileCoord& tc,
-                                                     uint32_t rank, int ew, int warp) {
-  const GroupDesc& gd = a.groups[tc.g];
-  const int row0 = tc.I * kPairTile + static_cast<int>(rank) * kHalf + (warp & 3) * 32;
-  if (row0 >= gd.r) return;
-  const int bz = static_cast<int>(tc.b);
-  const int mat = gd.first_mat + bz;
-  const MatDesc& md = a.mats[mat];
-  const bool w_tma = md.W && last_by_tma(md);
-  const int ch_begin = (ew / 4) * L::kChunksPerWarp;
-  for (int ch = ch_begin; ch < ch_begin + L::kChunksPerWarp; ++ch) {
-    const int col0 = tc.J * kPairTile + ch * 32;
-    if (col0 >= gd.c) break;
-    ptx::tma_prefetch_3d(tmap(a, tc.g, kTmXloE), col0, row0, bz);
-    if (w_tma)
-      ptx::tma_prefetch_3d(mat_tmap(a, mat, kMtW), md.transposed ? row0 : col0,
-                           md.transposed ? col0 : row0, 0);
-  }
-}
-
 // Epilogue warp: one tile. With `dep` set (chained launch) the warp first
 // waits until the tile's inputs have landed (counter >= need) and, once its
-// own stores have landed, adds one to the matrix's counter. `next` (the last
-// Apply) is the pair's next tile, whose inputs are prefetched into L2.
-// Returns false when a wait gives up (the pair has been aborted).
+// own stores have landed, adds one to the matrix's counter. Returns false
+// when a wait gives up (the pair has been aborted).
 template <int KIND, typename L>
 __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p, const Smem& s,
                                               const TileCoord& tc, int64_t t_apply, uint32_t rank,
                                               int ew, int warp, int lane, uint32_t tmem_base,
                                               EpiState& es, const uint32_t* leader_tempty,
-                                              uint64_t limit, unsigned* dep, uint32_t need,
-                                              const TileCoord* next = nullptr) {
+                                              uint64_t limit, unsigned* dep, uint32_t need) {
   using K = KindT<KIND>;
   const int quarter = warp & 3;  // TMEM lanes this warp may read: 32 * quarter ...
   const int ch_begin = (ew / 4) * L::kChunksPerWarp;  // this warp's share of the columns
@@ -737,7 +718,6 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
       ptx::bulk_wait_read<0>();  // the previous tile's stores have read every slot
       for (int ch = ch_begin; ch < ch_begin + D; ++ch)
         if (live_chunk(ch)) issue_load(ch);
-      if (KIND == kApplyLast && next != nullptr) prefetch_last_inputs<L>(a, *next, rank, ew, warp);
     }
   }
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -929,10 +909,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(StageLayout<KIND, WI
     bool ok = true;
     for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<KIND>(a, t);
-      const bool has_next = KIND == kApplyLast && t + npairs < a.total_tiles;
-      const TileCoord nx = has_next ? decode_tile<KIND>(a, t + npairs) : tc;
       ok = epilogue_tile<KIND, L>(a, p, s, tc, t, rank, ew, warp, lane, tmem_base, es, leader_tempty,
-                                  limit, nullptr, 0u, has_next ? &nx : nullptr);
+                                  limit, nullptr, 0u);
     }
     if (lane == 0) ptx::bulk_wait<0>();
     if (!ok) linger();

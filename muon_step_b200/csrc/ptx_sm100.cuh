@@ -229,14 +229,6 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_
       : "memory");
 }
 
-// Hint: bring a 3-D tile of the tensor map into L2 (no completion, no data in
-// shared memory). c0 follows the same 16-byte rule as the loads.
-__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N committed bulk groups still read shared memory.
