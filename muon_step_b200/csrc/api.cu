@@ -480,7 +480,7 @@ bool valid_shape(int64_t n, int64_t m) {
 // it depends on, with the other matrices' tiles in between, so CTA pairs that
 // reach it seldom wait; the window's buffers are the working set that stays
 // in L2. W defaults to the number of matrices whose average stage gives
-// every CTA pair three tiles per round, and at least two.
+// every CTA pair two and a half tiles per round, and at least two.
 void build_chain(const muon_plan_s* p, int npairs, ChainTile* out) {
   std::vector<int> mats;
   double stage_tiles = 0.0;
@@ -497,7 +497,7 @@ void build_chain(const muon_plan_s* p, int npairs, ChainTile* out) {
     // at least two, so that another matrix's tiles sit between a stage and
     // the stage that depends on it, covering the first one's last tiles
     const double mean = stage_tiles / static_cast<double>(mats.size());
-    window = std::max(2, static_cast<int>(std::ceil(3.0 * std::max(npairs, 1) / std::max(mean, 1.0))));
+    window = std::max(2, static_cast<int>(std::ceil(2.5 * std::max(npairs, 1) / std::max(mean, 1.0))));
   }
   window = std::max(1, std::min<int>(window, static_cast<int>(mats.size())));
   const int nstages = 3 * p->steps;

@@ -367,7 +367,7 @@ def build_chain(shapes, npairs, steps=10, window=0):
         return groups, per, mats, []
     if window <= 0:
         mean = sum(sum(per[mats[k][0]]) / 3.0 for k in grouped) / len(grouped)
-        window = max(2, math.ceil(3.0 * max(npairs, 1) / max(mean, 1.0)))
+        window = max(2, math.ceil(2.5 * max(npairs, 1) / max(mean, 1.0)))
     window = max(1, min(window, len(grouped)))
     out, act, nxt = [], [], 0
     while nxt < len(grouped) or act:
