@@ -171,16 +171,15 @@ MUON_API muon_status_t muon_plan_set_l2_batching(muon_plan_t plan, size_t bytes)
  * (without L2 batching). on = 1 (the default): every Gram, Poly and Apply
  * stage of the schedule in one persistent launch, then the last Apply fused
  * with the update. Its CTA pairs take the tiles of a host-built list in
- * order; a tile waits (bounded) until the earlier stages of its own matrix
- * have finished, signalled through per-matrix counters in the workspace. The
- * list keeps `window` matrices in flight at a time (0: chosen from the tile
- * counts), so their buffers can stay in L2 from one stage to the next.
- * on = 0: one launch per stage and step. Both give bit-identical results.
- * The chained launch sizes its grid so that all its CTA pairs are resident
- * at once on an otherwise idle GPU; work of other streams that occupies SMs
- * when it starts can hold some pairs back, and the bounded waits then report
- * MUON_ERR_TIMEOUT (use on = 0 in that setting). Timing events must be set
- * again afterwards. */
+ * order, each pair the next unclaimed one (a counter in the workspace) as it
+ * becomes free; a tile waits (bounded) until the earlier stages of its own
+ * matrix have finished, signalled through per-matrix counters in the
+ * workspace. The list keeps `window` matrices in flight at a time (0: chosen
+ * from the tile counts), so their buffers can stay in L2 from one stage to
+ * the next. on = 0: one launch per stage and step. Both give bit-identical
+ * results. Pairs that other streams' work keeps from starting delay the
+ * chained launch but cannot stall it. Timing events must be set again
+ * afterwards. */
 MUON_API muon_status_t muon_plan_set_chaining(muon_plan_t plan, int on, int window);
 
 /* Bytes of workspace the plan needs (device memory, 256-byte aligned). */

@@ -415,7 +415,7 @@ muon_status_t build_plan(muon_plan_s* p, const std::vector<MatDesc>& caller) {
   p->off_chain = off;
   off = align_up(off + static_cast<size_t>(p->chain_len) * sizeof(ChainTile), 256);
   p->off_dep = off;
-  off = align_up(off + (tc ? nm * sizeof(unsigned) : 0), 256);
+  off = align_up(off + (tc ? (nm + 1) * sizeof(unsigned) : 0), 256);  // + the tile counter
   p->desc_bytes = off;
   off = align_up(off, 1024);
   for (auto& gd : p->groups) {
@@ -757,6 +757,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
   ew.eps = plan->eps;
   ew.diag = plan->mode == 0 ? plan->diag : nullptr;
   ew.dep = chained(plan) ? reinterpret_cast<unsigned*>(ws + plan->off_dep) : nullptr;
+  ew.next_tile = ew.dep ? ew.dep + plan->mats.size() : nullptr;
   if ((st = record(plan, 0, stream)) != MUON_OK) return st;
   if (launch_elementwise(ew, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if ((st = record(plan, 1, stream)) != MUON_OK) return st;
@@ -871,6 +872,7 @@ muon_status_t muon_plan_execute(muon_plan_t plan, const muon_hyper_t* hyper, voi
     sa.total_tiles = plan->chain_len;
     sa.chain = reinterpret_cast<const ChainTile*>(ws + plan->off_chain);
     sa.dep = reinterpret_cast<unsigned*>(ws + plan->off_dep);
+    sa.next_tile = sa.dep + plan->mats.size();
     sa.chain_stages = unit ? 3 * plan->steps : 3 * plan->steps - 1;
     sa.last = 0;
     if (unit) {

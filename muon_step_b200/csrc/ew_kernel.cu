@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(kEwThreads, kEwMinBlocks) ew_kernel(const __gr
   const GroupDesc& gd = a.groups[md.group];
   const int64_t n = md.n, m = md.m;
   const int64_t ldc = gd.ldc;
+  if (a.next_tile && tile == 0 && tid == 0) *a.next_tile = 0u;  // the chained launch's list starts over
   const int gr = gd.r;
   const int lo_kind = gd.small;  // layout of the low part (lo_index)
 

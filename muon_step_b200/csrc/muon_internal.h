@@ -138,6 +138,7 @@ struct StageArgs {
   // persistent kernel, tiles taken in the order of a host-built list
   const ChainTile* chain; // [total_tiles]
   unsigned* dep;          // per matrix: epilogue-warp tile completions so far this execute
+  unsigned* next_tile;    // the list index the next CTA pair to ask takes (zero at launch)
   int32_t chain_sumsq_stage;  // stage whose Apply records sums of squares (-1: none)
   int32_t chain_stages;       // tiles of later stages in the list are skipped
   float abc[kMaxSteps * 3];   // every step's coefficients
@@ -161,6 +162,7 @@ struct EwArgs {
   float mu, eps;
   float* diag;            // optional: diag[2 caller] = ||N||_F
   unsigned* dep;          // optional: chained-launch dependency counters, reset per matrix
+  unsigned* next_tile;    // optional: chained-launch tile counter, reset by the first CTA
 };
 
 // Small-matrix kernel arguments (one CTA per matrix, every step on chip).

@@ -65,9 +65,13 @@
 //                          landed: wait, proxy fence, release add), and a
 //                          tile's producer and epilogue warps wait (acquire)
 //                          until every tile of the matrix's earlier stages
-//                          has finished. Every CTA pair takes its tiles in
-//                          list order and all pairs are resident at once,
-//                          so the earliest unfinished tile can always run.
+//                          has finished. CTA pairs take list indices from
+//                          a global counter as they become free (the pair
+//                          leader's producer fetches and publishes each to
+//                          both CTAs' roles through a small queue), so the
+//                          earliest unfinished tile is always held by a
+//                          running pair and can run, however many pairs the
+//                          device holds at once.
 //
 // Every spin-wait is bounded; on expiry the kernel raises the error word and
 // an abort flag in both CTAs, stops issuing work, drains what is in flight,
@@ -96,6 +100,7 @@ constexpr int kEpiF32 = 32 * 32 * 4;              // fp32 32 x 32, 128-byte swiz
 constexpr int kEpiB16 = 32 * 32 * 2;              // bf16 32 x 32, 64-byte swizzle
 constexpr size_t kBarrierBytes = 512;
 constexpr int kTmapBytes = 128;
+constexpr int kTileQ = 4;  // chained launch: tile indices published ahead of their use
 
 // Facts of a tile kind that do not depend on the launch layout. Slot use:
 //   Gram       [bf16 out | bf16 mirror out]                            4 KB
@@ -126,6 +131,10 @@ struct Layout {
   static constexpr int kEpiBytes = EPI_WARPS * SLOTS * SLOT;
   static constexpr size_t kSmem = 1024 + STAGES * kStageBytes + kEpiBytes + kBarrierBytes;
   static constexpr int kChunksPerWarp = (kPairTile / 32) / (EPI_WARPS / 4);
+  // mbarriers (ring, accumulators, drain, epilogue loads, tile queue), then
+  // the TMEM address, the abort flag and the tile queue's entries
+  static_assert(8 * (2 * STAGES + 5 + SLOTS * EPI_WARPS + 2 * kTileQ) + 8 + 4 * kTileQ <= kBarrierBytes,
+                "barrier area");
 };
 
 // Layout of the one-stage kernels. Wide variants run eight epilogue warps
@@ -288,8 +297,11 @@ struct Smem {
   uint64_t* tempty;
   uint64_t* drain;
   uint64_t* eload;  // epilogue warps x slots
+  uint64_t* tq_full;   // chained launch: tile queue, entry published (both CTAs)
+  uint64_t* tq_empty;  // ... entry read by every consumer (pair leader)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
+  volatile uint32_t* tq;  // tile indices
 };
 
 template <typename L>
@@ -305,8 +317,11 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
   s.eload = s.drain + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.eload + L::kEpiSlots * L::kEpiWarps);
+  s.tq_full = s.eload + L::kEpiSlots * L::kEpiWarps;
+  s.tq_empty = s.tq_full + kTileQ;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.tq_empty + kTileQ);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
+  s.tq = reinterpret_cast<volatile uint32_t*>(s.abort_flag + 1);
   return s;
 }
 
@@ -812,6 +827,12 @@ __device__ __forceinline__ uint32_t prologue(const Smem& s, int warp) {
     }
     ptx::mbar_init(s.drain, 1);
     for (int i = 0; i < L::kEpiSlots * L::kEpiWarps; ++i) ptx::mbar_init(&s.eload[i], 1);
+    // chained launch's tile queue: published by the leader's producer; read by
+    // the leader's MMA warp, the peer's producer and both CTAs' epilogue warps
+    for (int i = 0; i < kTileQ; ++i) {
+      ptx::mbar_init(&s.tq_full[i], 1);
+      ptx::mbar_init(&s.tq_empty[i], 2 + 2 * L::kEpiWarps);
+    }
     *s.abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -919,6 +940,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(StageLayout<KIND, WI
   teardown(warp, tmem_base);
 }
 
+// The chained launch's tile queue. The pair leader's producer takes the next
+// tile index from the global counter and publishes it to both CTAs; every
+// other role of the pair takes the indices from its CTA's queue in the same
+// order. An index at or past the end of the list ends every role's loop.
+struct TileQueue {
+  uint32_t slot = 0, phase = 0;
+  __device__ void advance() {
+    if (++slot == kTileQ) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+};
+
+// Leader producer: fetch, then publish to both CTAs (the queue entry must
+// have been read by all consumers of its previous use).
+__device__ __forceinline__ bool tq_publish(const StageArgs& a, const Smem& s, TileQueue& q, uint64_t limit,
+                                           uint32_t& t) {
+  t = atomicAdd(a.next_tile, 1u);
+  if (!ptx::mbar_wait_cluster(&s.tq_empty[q.slot], q.phase ^ 1, limit, s.abort_flag)) return false;
+  const uint32_t entry = ptx::smem_u32(const_cast<uint32_t*>(s.tq + q.slot));
+  const uint32_t full = ptx::smem_u32(&s.tq_full[q.slot]);
+  for (uint32_t r = 0; r < 2; ++r) {
+    ptx::st_cluster_u32(ptx::mapa_shared(entry, r), t);
+    ptx::mbar_arrive_release_cluster(ptx::mapa_shared(full, r));
+  }
+  q.advance();
+  return true;
+}
+
+// Any other role: the next published index of this CTA's queue.
+__device__ __forceinline__ bool tq_take(const Smem& s, TileQueue& q, uint64_t limit, uint32_t& t) {
+  if (!ptx::mbar_wait_cluster(&s.tq_full[q.slot], q.phase, limit, s.abort_flag)) return false;
+  t = s.tq[q.slot];
+  ptx::mbar_arrive_release_cluster(ptx::mapa_shared(ptx::smem_u32(&s.tq_empty[q.slot]), 0));
+  q.advance();
+  return true;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
     stage_chain_kernel(const __grid_constant__ StageArgs a) {
   using L = ChainL;
@@ -927,9 +987,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
-  const int64_t pair = blockIdx.x >> 1;
-  const int64_t npairs = gridDim.x >> 1;
   const uint64_t limit = a.wait_limit_ns;
+  const uint32_t total = static_cast<uint32_t>(a.total_tiles);
   const uint32_t tmem_base = prologue<L>(s, warp);
 
   if (warp == 0 && lane == 0) {
@@ -937,8 +996,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
     uint32_t leader_full[L::kStages];
     load_tmaps_and_full<L>(a, s, leader_full);
     uint32_t stage = 0, phase = 0;
+    TileQueue q;
     bool ok = true;
-    for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
+    for (;;) {
+      uint32_t t = 0;
+      if (!(rank == 0 ? tq_publish(a, s, q, limit, t) : tq_take(s, q, limit, t))) {
+        raise_abort(a, s);
+        ok = false;
+        break;
+      }
+      if (t >= total) break;
       const ChainTile ct = a.chain[t];
       if (ct.stage >= a.chain_stages) continue;  // skipped by every role of the pair
       const ChainPos cp = chain_pos(a, ct);
@@ -956,6 +1023,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
       if (!r) {
         raise_abort(a, s);
         ok = false;
+        break;
       }
     }
     if (!ok) linger();
@@ -963,13 +1031,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
     // ---------------------------------------------------------- MMA issuer (pair leader)
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
     bool issued = false;
-    for (int64_t t = a.tile_begin + pair; t < a.total_tiles; t += npairs) {
-      const ChainTile ct = a.chain[t];
-      if (ct.stage >= a.chain_stages) continue;
-      const ChainPos cp = chain_pos(a, ct);
-      bool r;
-      if (cp.kind == kApply) r = mma_tile<kApply, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
-      else r = mma_tile<kGram, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
+    TileQueue q;
+    for (;;) {
+      uint32_t t = 0;
+      bool r = tq_take(s, q, limit, t);
+      if (r && t >= total) break;
+      if (r) {
+        const ChainTile ct = a.chain[t];
+        if (ct.stage >= a.chain_stages) continue;
+        const ChainPos cp = chain_pos(a, ct);
+        if (cp.kind == kApply) r = mma_tile<kApply, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
+        else r = mma_tile<kGram, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
+      }
       if (!r) {
         raise_abort(a, s);
         if (issued) drain_mma(s, limit);
@@ -982,8 +1055,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
     uint32_t leader_tempty[2];
     for (int i = 0; i < 2; ++i) leader_tempty[i] = ptx::mapa_shared(ptx::smem_u32(&s.tempty[i]), 0);
     EpiState es;
+    TileQueue q;
     bool ok = true;
-    for (int64_t t = a.tile_begin + pair; ok && t < a.total_tiles; t += npairs) {
+    for (;;) {
+      uint32_t t = 0;
+      int took = 1;
+      if (lane == 0) took = tq_take(s, q, limit, t) ? 1 : 0;
+      else q.advance();  // every lane follows the queue position (lane 0 reads it)
+      took = __shfl_sync(0xffffffffu, took, 0);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!took) {
+        if (lane == 0) raise_abort(a, s);
+        ok = false;
+        break;
+      }
+      if (t >= total) break;
       const ChainTile ct = a.chain[t];
       if (ct.stage >= a.chain_stages) continue;
       const ChainPos cp = chain_pos(a, ct);
@@ -997,6 +1083,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
       else
         ok = epilogue_tile<kApply, L>(a, p, s, cp.tc, cp.t_apply, rank, ew, warp, lane, tmem_base, es,
                                       leader_tempty, limit, a.dep, cp.need);
+      if (!ok) break;
     }
     if (lane == 0) ptx::bulk_wait<0>();
     if (!ok) linger();

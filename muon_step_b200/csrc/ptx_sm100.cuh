@@ -347,3 +347,43 @@ __device__ __forceinline__ bool dep_wait(const unsigned* ctr, uint32_t target, c
 
 }  // namespace ptx
 }  // namespace muon
+
+namespace muon {
+namespace ptx {
+
+// ---------------------------------------------------------------- mbarriers across the CTA pair
+// Arrive on an mbarrier of either CTA of the cluster (shared::cluster address),
+// releasing this thread's earlier writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with acquire at cluster scope (for phases completed by arrivals
+// from the other CTA of the pair).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                  volatile int* abort_flag) {
+  if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint64_t it = 0; it < kSpinBackstop; ++it) {
+    if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if ((it & 15) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return false;
+}
+
+}  // namespace ptx
+}  // namespace muon

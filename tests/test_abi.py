@@ -157,7 +157,8 @@ def expected_workspace(shapes, prec):
     off = al(off + apply_tiles * slots * 4, 256)
     off = al(off + nm * 4, 256)
     # chained launch (bf16): a 16-byte entry per tile of every stage of every
-    # step of every grouped matrix, then a dependency counter per matrix
+    # step of every grouped matrix, then a dependency counter per matrix and
+    # the tile counter
     if prec == MUON_NS_BF16:
         chain = 0
         for (r, c), mem in groups.items():
@@ -165,7 +166,7 @@ def expected_workspace(shapes, prec):
                 pb = math.ceil(r / 256)
                 chain += len(mem) * 10 * (2 * (pb * (pb + 1) // 2) + pb * math.ceil(c / 256))
         off = al(off + chain * 16, 256)
-        off = al(off + nm * 4, 256)
+        off = al(off + (nm + 1) * 4, 256)
     off = al(off, 1024)
     for (r, c), mem in sorted(groups.items(), key=lambda kv: order.index(kv[0])):
         k = len(mem)

@@ -390,29 +390,36 @@ def chain_need(per_g, stage):
     return CHAIN_ARRIVALS * (step * (g0 + p0 + a0) + (g0 if kind >= 1 else 0) + (p0 if kind >= 2 else 0))
 
 
-def simulate_chain(shapes, npairs, steps=10, window=0, chain_stages=None):
-    """Every pair takes its tiles (t = pair, pair + npairs, ...) in list order;
-    a tile starts when its matrix's counter has reached its target and adds
-    CHAIN_ARRIVALS when it finishes (its time: its K blocks). Returns the
-    makespan; fails on a deadlock."""
+def simulate_chain(shapes, npairs, steps=10, window=0, chain_stages=None, resident=None):
+    """CTA pairs take list indices from one shared counter, in increasing order,
+    as they become free (an index of a skipped stage is taken and dropped); a
+    pair holding a tile starts it when its matrix's counter has reached the
+    target and adds CHAIN_ARRIVALS when it finishes (its time: its K blocks).
+    Only `resident` of the launch's pairs ever run (default: all), as when the
+    device cannot hold the whole grid at once. Returns the makespan; fails on
+    a deadlock."""
     groups, per, mats, tiles = build_chain(shapes, npairs, steps, window)
     nst = 3 * steps if chain_stages is None else chain_stages
+    run = npairs if resident is None else resident
     dep = [0] * len(mats)
-    pos = [p for p in range(npairs)]        # next list index of each pair
-    busy = [0.0] * npairs                   # time each pair becomes free
+    nxt = 0                                 # the shared tile counter
+    held = [None] * run                     # list index a pair has taken
+    busy = [0.0] * run                      # time each pair becomes free
     now, done, running = 0.0, 0, []         # running: (finish time, pair, matrix)
     todo = sum(1 for _, s, _ in tiles if s < nst)
     import heapq
     while done < todo:
         progressed = False
-        for p in range(npairs):
+        for p in range(run):
             if busy[p] > now:
                 continue
-            while pos[p] < len(tiles) and tiles[pos[p]][1] >= nst:
-                pos[p] += npairs            # skipped by every role
-            if pos[p] >= len(tiles):
+            while held[p] is None and nxt < len(tiles):
+                if tiles[nxt][1] < nst:
+                    held[p] = nxt
+                nxt += 1                    # skipped indices are dropped by every role
+            if held[p] is None:
                 continue
-            mat, stage, u = tiles[pos[p]]
+            mat, stage, u = tiles[held[p]]
             g = mats[mat][0]
             if dep[mat] < chain_need(per[g], stage):
                 continue
@@ -421,7 +428,7 @@ def simulate_chain(shapes, npairs, steps=10, window=0, chain_stages=None):
             t_end = now + cdiv(k, BK)
             heapq.heappush(running, (t_end, p, mat))
             busy[p] = t_end
-            pos[p] += npairs
+            held[p] = None
             progressed = True
         if running:
             t_end, p, mat = heapq.heappop(running)
@@ -464,6 +471,18 @@ def test_chain_list_covers_every_stage_once_and_never_deadlocks(shapes, npairs):
             for i, (mat, stage, u) in enumerate(tiles):
                 if stage > 0:
                     assert first_pos[(mat, stage - 1)] < first_pos[(mat, stage)] <= i
+
+
+@pytest.mark.parametrize("resident", [1, 2, 37])
+def test_chain_finishes_with_any_number_of_resident_pairs(resident):
+    """Tiles go to whichever pair asks next, so the list completes even when
+    the device runs fewer pairs at once than the launch has (the rest start
+    later or, here, never)."""
+    shapes = [(1024, 1024)] * 12 + [(512, 2048)] * 3
+    full, dep, per, mats, _ = simulate_chain(shapes, 74)
+    t, dep_r, _, _, _ = simulate_chain(shapes, 74, resident=resident)
+    assert dep_r == dep
+    assert t >= full
 
 
 def test_chain_targets_are_prefix_sums_of_earlier_stages():
