@@ -518,3 +518,36 @@ def test_chained_orthogonalize_matches_stagewise():
     assert ms.sync_status() == 0
     for oa, ob in zip(*outs):
         assert torch.equal(oa, ob)
+
+
+def test_chained_launch_beside_work_on_another_stream():
+    """The chained launch's CTA pairs take tiles from a shared counter as they
+    become free, so matrix products running on another stream when it starts
+    (holding SMs it would use) only delay it: no timeout, and the same bits
+    as the per-stage launches on an otherwise idle GPU."""
+    import muon_step_b200 as ms
+
+    shapes = [(1024, 1024)] * 6 + [(512, 2048), (2048, 512), (600, 600)]
+    a = workloads.make_random(shapes, device="cuda", seed=89)
+    b = workloads.make_random(shapes, device="cuda", seed=89)
+    pa = ms.MuonPlan([(a.W[k], a.G[k], a.M[k]) for k in range(a.count)])
+    pb = ms.MuonPlan([(b.W[k], b.G[k], b.M[k]) for k in range(b.count)])
+    pa.set_chaining(True)
+    pb.set_chaining(False)
+    wa = pa.alloc_workspace()
+    x = torch.randn(8192, 8192, device="cuda", dtype=torch.bfloat16)
+    other = torch.cuda.Stream()
+    mine = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        with torch.cuda.stream(other):
+            for _ in range(8):
+                y = x @ x
+        pa.execute(wa, stream=mine)
+        pb.execute()
+    torch.cuda.synchronize()
+    del y
+    assert ms.sync_status() == 0
+    for k in range(a.count):
+        assert torch.equal(a.W[k], b.W[k]), k
+        assert torch.equal(a.M[k], b.M[k]), k
