@@ -13,14 +13,16 @@
 //                  of the Gram product and, read as 64-column chunks, the
 //                  MN-major operand of the Apply product; A and B as 128 x 128
 //                  bf16 tiles (64 KB).
-//   global (L2)    the iterate's bf16 low part, read and rewritten in place by
-//                  the thread that owns each element (iterate = high + low).
-//   TMEM           all 512 columns: the 128 x 128 accumulators of the Gram
-//                  and Poly products, the 128 x c accumulator of the Apply
-//                  product (two N = 256 instructions).
+//   TMEM           columns 0 .. 255: the 128 x 128 accumulators of the Gram
+//                  and Poly products and, one column half at a time, the
+//                  128 x 256 accumulator of the Apply product (one N = 256
+//                  instruction per K = 16); columns 256 .. 511: the iterate's
+//                  bf16 low part (iterate = high + low), two elements a
+//                  column, loaded from global memory once per matrix and
+//                  rewritten in place by each Apply epilogue.
 //
 // Thread t owns iterate row t % 128 (its TMEM lane) and column quarter t / 128:
-// 32 columns of A and B, 128 columns of X. The elementwise kernel has written
+// 32 columns of A and B; in each Apply half, 64 columns of X. The elementwise kernel has written
 // N as high + low parts and the scale s; step one folds s^2 into A and s into
 // X'. After the last step the update W <- W (1 - lr wd) - lr gamma
 // sqrt(max(n, m)) O' ("Muon 优化器完全拆解…", Algorithm 1 steps four and five, or
@@ -45,6 +47,7 @@ constexpr int kTileBytes = 2 * kChunkBytes;         // 128 x 128 bf16
 constexpr int kThreads = 512;
 constexpr size_t kSmem = 1024 + kXBytes + 2 * kTileBytes + 64;
 constexpr int kTmemCols = 512;
+constexpr int kLoCol = 256;  // TMEM columns 256 .. 511: the iterate's low part, two bf16 a column
 constexpr uint32_t kIdescKK = ptx::idesc_bf16(kR, kR, 0, 0);   // M = N = 128, both K-major
 constexpr uint32_t kIdescApply = ptx::idesc_bf16(kR, 256, 0, 1);  // M = 128, N = 256, B MN-major
 
@@ -77,21 +80,53 @@ __device__ __forceinline__ void gemm_poly(uint32_t d, uint32_t sa) {
   }
 }
 
-// D[:, 256 h ..] = B X[:, 256 h ..] over K = 128 for the nh column halves.
-__device__ __forceinline__ void gemm_apply(uint32_t d, uint32_t sb, uint32_t sx, int nh) {
-  for (int h = 0; h < nh; ++h) {
+// D[:, 0 .. 256) = B X[:, 256 h ..] over K = 128: column half h of the Apply
+// product (one N = 256 instruction per K = 16).
+__device__ __forceinline__ void gemm_apply_half(uint32_t d, uint32_t sb, uint32_t sx, int h) {
 #pragma unroll
-    for (int k = 0; k < kR / 16; ++k) {
-      const uint64_t ad = ptx::desc_sw128(sb + (k >> 2) * kChunkBytes + (k & 3) * 32, 16, 1024);
-      const uint64_t bd = ptx::desc_sw128(sx + h * 4 * kChunkBytes + k * 16 * 128, kChunkBytes, 1024);
-      ptx::umma_bf16(d + h * 256, ad, bd, kIdescApply, k != 0);
-    }
+  for (int k = 0; k < kR / 16; ++k) {
+    const uint64_t ad = ptx::desc_sw128(sb + (k >> 2) * kChunkBytes + (k & 3) * 32, 16, 1024);
+    const uint64_t bd = ptx::desc_sw128(sx + h * 4 * kChunkBytes + k * 16 * 128, kChunkBytes, 1024);
+    ptx::umma_bf16(d, ad, bd, kIdescApply, k != 0);
   }
 }
 
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+// tcgen05.ld / tcgen05.st of 16 consecutive 32-bit TMEM columns of this
+// warp's 32 lanes (one row per thread).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
+  __nv_bfloat162 b;
+  memcpy(&b, &u, 4);
+  return b;
+}
+
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 b) {
+  uint32_t u;
+  memcpy(&u, &b, 4);
+  return u;
+}
+
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -108,28 +143,22 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int i, int ch, const fl
 }
 
 // One 32-column chunk of the Apply epilogue for iterate row `row`:
-// X' = alpha (a X + v) with X = high (shared) + low (global), written back as
-// high and low parts. kFirst folds alpha (step one), kLast accumulates the
-// sum of squares, kMask zeroes what lies outside the matrix (ragged chunks).
+// X' = alpha (a X + v) with X = high (shared) + low (`lw`: word i holds
+// columns col0 + 2 i and col0 + 2 i + 1), written back as high and low parts.
+// kFirst folds alpha (step one), kLast accumulates the sum of squares, kMask
+// zeroes what lies outside the matrix (ragged chunks).
 template <bool kFirst, bool kLast, bool kMask>
-__device__ __forceinline__ void apply_chunk(uint8_t* Xs, __nv_bfloat16* xl, int row, int col0, int r,
-                                            int c, bool row_in, float alpha, float ca,
-                                            const float (&v)[32], float& ssq) {
+__device__ __forceinline__ void apply_chunk(uint8_t* Xs, int row, int col0, int c, bool row_in, float alpha,
+                                            float ca, const float (&v)[32], uint32_t (&lw)[16], float& ssq) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int p = col0 / 8 + q;
     Bf16x8 h8 = *reinterpret_cast<const Bf16x8*>(Xs + piece_off(row, p));
-    const bool grp = !kMask || (row_in && col0 + 8 * q < c);  // 8 columns that start inside
-    __nv_bfloat16* lp = xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8;
-    uint4 lraw = make_uint4(0u, 0u, 0u, 0u);
-    if (grp) lraw = *reinterpret_cast<const uint4*>(lp);
-    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lraw);
-    Bf16x8 lo8;
 #pragma unroll
     for (int hh = 0; hh < 4; ++hh) {
       const int e = 8 * q + 2 * hh;
       const float2 fh = __bfloat1622float2(h8.v[hh]);
-      const float2 fl = __bfloat1622float2(l2[hh]);
+      const float2 fl = __bfloat1622float2(as_bf2(lw[4 * q + hh]));
       float x0 = fh.x + fl.x, x1 = fh.y + fl.y;
       if (kMask) {
         // columns c .. ldc of the low part are not written by the elementwise kernel
@@ -144,28 +173,34 @@ __device__ __forceinline__ void apply_chunk(uint8_t* Xs, __nv_bfloat16* xl, int 
       if (kLast) ssq = fmaf(y0, y0, fmaf(y1, y1, ssq));
       h8.v[hh] = __floats2bfloat162_rn(y0, y1);
       const float2 nh2 = __bfloat1622float2(h8.v[hh]);
-      lo8.v[hh] = __floats2bfloat162_rn(y0 - nh2.x, y1 - nh2.y);
+      lw[4 * q + hh] = as_u32(__floats2bfloat162_rn(y0 - nh2.x, y1 - nh2.y));
     }
     *reinterpret_cast<Bf16x8*>(Xs + piece_off(row, p)) = h8;
-    if (grp) *reinterpret_cast<Bf16x8*>(lp) = lo8;
   }
 }
 
+// The epilogue of column half h: thread quarter cq takes iterate columns
+// 256 h + 64 cq .. + 63 (two chunks); the accumulator holds the half at TMEM
+// columns 0 .. 255, the low part sits at column kLoCol + col / 2.
 template <bool kFirst, bool kLast>
-__device__ __forceinline__ void apply_epilogue(uint8_t* Xs, __nv_bfloat16* xl, uint32_t trow, int row,
-                                               int cq, int r, int c, bool row_in, float alpha,
-                                               float ca, float& ssq) {
-#pragma unroll 1
-  for (int j = 0; j < 4; ++j) {
-    const int col0 = 128 * cq + 32 * j;
-    if (col0 >= c) break;  // the same for the whole warp
+__device__ __forceinline__ void apply_epilogue(uint8_t* Xs, uint32_t trow, int row, int cq, int h, int c,
+                                               bool row_in, float alpha, float ca, float& ssq) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int acc = 64 * cq + 32 * j;  // accumulator column
+    const int col0 = 256 * h + acc;    // iterate column
+    if (col0 >= c) break;              // the same for the whole warp
     float v[32];
-    ptx::tmem_ld32(trow + col0, v);
+    uint32_t lw[16];
+    ptx::tmem_ld32(trow + acc, v);
+    tmem_ld16(trow + kLoCol + (col0 >> 1), lw);
     if (row_in && col0 + 32 <= c)
-      apply_chunk<kFirst, kLast, false>(Xs, xl, row, col0, r, c, row_in, alpha, ca, v, ssq);
+      apply_chunk<kFirst, kLast, false>(Xs, row, col0, c, row_in, alpha, ca, v, lw, ssq);
     else
-      apply_chunk<kFirst, kLast, true>(Xs, xl, row, col0, r, c, row_in, alpha, ca, v, ssq);
+      apply_chunk<kFirst, kLast, true>(Xs, row, col0, c, row_in, alpha, ca, v, lw, ssq);
+    tmem_st16(trow + kLoCol + (col0 >> 1), lw);
   }
+  tmem_wait_st();
 }
 
 }  // namespace
@@ -244,6 +279,26 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
     __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(a.ws + gd.xlo_off) +
                         static_cast<int64_t>(md.index) * r * ldc + static_cast<int64_t>(row) * 8;
     const bool row_in = row < r;
+    // the low part into TMEM columns kLoCol + col / 2: this thread's row,
+    // columns 128 cq .. 128 cq + 127 (8-column groups past the matrix: zero)
+    ptx::tc_fence_after();
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      const int col0 = 128 * cq + 32 * g;
+      uint32_t lw[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 lraw = make_uint4(0u, 0u, 0u, 0u);
+        if (row_in && col0 + 8 * q < c)
+          lraw = *reinterpret_cast<const uint4*>(xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8);
+        lw[4 * q] = lraw.x;
+        lw[4 * q + 1] = lraw.y;
+        lw[4 * q + 2] = lraw.z;
+        lw[4 * q + 3] = lraw.w;
+      }
+      tmem_st16(trow + kLoCol + (col0 >> 1), lw);
+    }
+    tmem_wait_st();
     if (!ptx::mbar_wait(bar_ld, ld_phase, limit, abort_flag)) {
       *abort_flag = 1;
       atomicOr(a.err, kErrTimeout);
@@ -300,34 +355,33 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
       }
       hand_over();
 
-      // Apply: X' = alpha (a X + B X), X = high (shared) + low (global)
-      if (tid == 0) {
-        ptx::tc_fence_after();
-        gemm_apply(tmem, sB, sX, nh);
-        ptx::umma_commit(bar_mma);
-      }
+      // Apply: X' = alpha (a X + B X), X = high (shared) + low (TMEM), one
+      // column half at a time: the product of half 1 reads X columns 256 ..
+      // only, which the epilogue of half 0 leaves alone
       const bool last = (k + 1 == a.steps);
-      // while the product runs: this thread's low-part pieces into L1, and on
-      // the last step the caller's weight into L2 for the update
-      if (row_in) {
-        for (int g = 16 * cq; g < 16 * cq + 16 && 8 * g < c; ++g)
-          prefetch_l1(xl + static_cast<int64_t>(g) * r * 8);
-      }
       if (last && md.W) {
+        // the caller's weight into L2 for the update while the products run
         const int64_t lines = (md.n * md.m + 31) / 32;  // 128-byte lines of W
         for (int64_t ln = tid; ln < lines; ln += kThreads) prefetch_l2(md.W + ln * 32);
       }
-      wait_mma();
-      if (!ok) break;
-      // variants without the step-one scale, sums or masks where they are not needed
-      if (k == 0) {
-        if (last) apply_epilogue<true, true>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
-        else apply_epilogue<true, false>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
-      } else {
-        if (last) apply_epilogue<false, true>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
-        else apply_epilogue<false, false>(Xs, xl, trow, row, cq, r, c, row_in, alpha, ca, ssq);
+      for (int h = 0; ok && h < nh; ++h) {
+        if (tid == 0) {
+          ptx::tc_fence_after();
+          gemm_apply_half(tmem, sB, sX, h);
+          ptx::umma_commit(bar_mma);
+        }
+        wait_mma();
+        if (!ok) break;
+        // variants without the step-one scale, sums or masks where they are not needed
+        if (k == 0) {
+          if (last) apply_epilogue<true, true>(Xs, trow, row, cq, h, c, row_in, alpha, ca, ssq);
+          else apply_epilogue<true, false>(Xs, trow, row, cq, h, c, row_in, alpha, ca, ssq);
+        } else {
+          if (last) apply_epilogue<false, true>(Xs, trow, row, cq, h, c, row_in, alpha, ca, ssq);
+          else apply_epilogue<false, false>(Xs, trow, row, cq, h, c, row_in, alpha, ca, ssq);
+        }
+        hand_over();
       }
-      hand_over();
     }
     if (!ok) break;
 
@@ -361,23 +415,22 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
     // 128 x 128 fp32 tile in the A / B area, word (i, j) at i * 128 + (j ^ (i % 32)),
     // then each warp updates whole caller rows with contiguous accesses.
     float* T = reinterpret_cast<float*>(As);
+    ptx::tc_fence_after();  // the low part was last written by other warps
     const bool tr = md.transposed != 0;
     for (int p0 = 0; p0 < c; p0 += 128) {
       const int bw = (c - p0) < 128 ? (c - p0) : 128;  // block width
       const int col0 = p0 + 32 * cq;
-      if (col0 < c) {
+      if (col0 < c) {  // the same for the whole warp
+        uint32_t lw[16];
+        tmem_ld16(trow + kLoCol + (col0 >> 1), lw);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const Bf16x8 h8 = *reinterpret_cast<const Bf16x8*>(Xs + piece_off(row, col0 / 8 + q));
-          const bool grp = row_in && col0 + 8 * q < c;
-          uint4 lraw = make_uint4(0u, 0u, 0u, 0u);
-          if (grp) lraw = *reinterpret_cast<const uint4*>(xl + static_cast<int64_t>((col0 >> 3) + q) * r * 8);
-          const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lraw);
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) {
             const int e = 8 * q + 2 * hh;
             const float2 fh = __bfloat1622float2(h8.v[hh]);
-            const float2 fl = __bfloat1622float2(l2[hh]);
+            const float2 fl = __bfloat1622float2(as_bf2(lw[4 * q + hh]));
             const int jj = 32 * cq + e;  // column within the block
             T[row * 128 + (jj ^ (row & 31))] = (row_in && col0 + e < c) ? fh.x + fl.x : 0.f;
             T[row * 128 + ((jj + 1) ^ (row & 31))] = (row_in && col0 + e + 1 < c) ? fh.y + fl.y : 0.f;
@@ -449,8 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_mid_kernel(const __grid_consta
       }
       __syncthreads();  // the next block rewrites the staging tile
     }
-    // the next matrix loads X by TMA over what this one read
+    // the next matrix loads X by TMA over what this one read, and its low
+    // part into TMEM over what this one's update read
     ptx::fence_async_shared();
+    ptx::tc_fence_before();
     __syncthreads();
   }
 

@@ -322,6 +322,57 @@ def test_mid_kernel_low_part_layout_is_a_bijection_into_its_buffer(r, c):
         assert starts == list(range(starts[0], starts[0] + 8 * len(starts), 8))
 
 
+MID_TMEM_COLS, MID_LO_COL = 512, 256
+
+
+def mid_kernel_tmem_columns(c):
+    """ns_mid_kernel's TMEM use for a matrix of c columns (128 < c <= 512):
+    the Apply product runs one column half h at a time into accumulator
+    columns 0 .. 255; in the epilogue of half h, thread quarter cq takes the
+    32-column chunks 256 h + 64 cq + 32 j (j = 0, 1) that start inside the
+    matrix; the low part of iterate column col sits at column 256 + col / 2,
+    loaded by quarter cq for chunks 128 cq + 32 g and read by the update for
+    chunks p0 + 32 cq. Returns, per iterate column, the (half, accumulator
+    column, low column) the epilogue uses, and the low columns the load and
+    the update touch."""
+    nh = cdiv(c, 256)
+    epi = {}
+    for h in range(nh):
+        for cq in range(4):
+            for j in range(2):
+                acc = 64 * cq + 32 * j
+                col0 = 256 * h + acc
+                if col0 >= c:
+                    break
+                for e in range(32):
+                    epi.setdefault(col0 + e, []).append((h, acc + e, MID_LO_COL + (col0 >> 1) + e // 2))
+    loaded = {MID_LO_COL + ((128 * cq + 32 * g) >> 1) + w for cq in range(4) for g in range(4) for w in range(16)}
+    updated = {}
+    for p0 in range(0, c, 128):
+        for cq in range(4):
+            col0 = p0 + 32 * cq
+            if col0 < c:
+                for e in range(32):
+                    updated.setdefault(col0 + e, MID_LO_COL + (col0 >> 1) + e // 2)
+    return epi, loaded, updated
+
+
+@pytest.mark.parametrize("c", [129, 200, 256, 257, 300, 383, 384, 500, 512])
+def test_mid_kernel_tmem_columns(c):
+    epi, loaded, updated = mid_kernel_tmem_columns(c)
+    for col in range(c):
+        # each column of the matrix goes through the epilogue exactly once, in
+        # its own half, from an accumulator column below the low part
+        assert len(epi[col]) == 1, col
+        h, acc, lo = epi[col][0]
+        assert h == col // 256 and acc == col - 256 * h and 0 <= acc < MID_LO_COL
+        assert lo == MID_LO_COL + col // 2 < MID_TMEM_COLS
+        # the low column was loaded at the start of the matrix; the update
+        # reads the same column
+        assert lo in loaded and updated[col] == lo
+    assert all(MID_LO_COL <= x < MID_TMEM_COLS for x in loaded)
+
+
 def tiny_kernel_accesses(n, m):
     """ns_tiny_kernel: caller element e = crow * m + ccol maps to iterate
     (i, j) = (ccol, crow) when n > m else (crow, ccol); X lives at i * (c | 1) + j
