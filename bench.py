@@ -60,6 +60,8 @@ def parse_args():
                          "scaling)")
     ap.add_argument("--config", default="dense_d4096")
     ap.add_argument("--precision", choices=["bf16", "fp32"], default="bf16")
+    ap.add_argument("--scale-mode", choices=["shape", "unit_rms", "none"], default="shape",
+                    help="update scale: sqrt(max(n, m)) gamma (default), unit RMS times gamma, or none")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
     ap.add_argument("--stagewise", action="store_true",
@@ -674,7 +676,7 @@ def main():
     wl = workloads.make(args.config, device=dev, **count_kwargs(args.config, args.count))
     h = wl.hyper
     params = [(wl.W[k], wl.G[k], wl.M[k]) for k in range(wl.count)]
-    plan = ms.MuonPlan(params, precision=args.precision)
+    plan = ms.MuonPlan(params, precision=args.precision, scale_mode=args.scale_mode)
     plan.set_chaining(not args.stagewise, args.chain_window)
     ws = plan.alloc_workspace()
     kinds = plan.launches()
@@ -856,6 +858,7 @@ def main():
             "config": {"workload": args.config, "matrices": wl.count,
                        "shapes": sorted({f"{n}x{m}" for n, m in wl.shapes}),
                        "ns_steps": ns_steps, "precision": args.precision,
+                       "scale_mode": args.scale_mode,
                        "l2": "inputs larger than L2 (no flush)" if wl.elements() * 12 > 126e6
                              else "inputs smaller than L2",
                        "metric_flops_per_step": flops_rank},
