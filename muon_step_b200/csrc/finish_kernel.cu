@@ -16,7 +16,12 @@
 //                       shared memory so every global access stays coalesced.
 //
 // HBM-bound: 4 B of O' read (fp32, or bf16 high + low parts), 8 B of W read
-// and written per element.
+// and written per element. Where the caller's rows allow 16-byte accesses
+// and the iterate is not transposed, a thread takes four consecutive columns
+// (one 16-byte piece of W, two 8-byte pieces of O') of eight rows, loading
+// four rows before it stores any, as the elementwise kernel does. (Transposed
+// tiles keep one column per thread: four-column reads of the staged tile
+// would meet four-way bank conflicts.)
 //
 // With diagnostics on, rms_reduce_kernel also runs after a fused last step (any
 // scale mode) and writes the RMS of the applied update per matrix.
@@ -60,7 +65,7 @@ __global__ void __launch_bounds__(256) rms_reduce_kernel(const __grid_constant__
   }
 }
 
-__global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ FinishArgs a) {
+__global__ void __launch_bounds__(256, 4) finish_kernel(const __grid_constant__ FinishArgs a) {
   __shared__ float stage[kEwRows][kEwCols + 1];
   const int tid = threadIdx.x;
   const int64_t tile = blockIdx.x;
@@ -83,6 +88,57 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
     return a.split ? __bfloat162float(oh[k]) + __bfloat162float(ol[k]) : of[k];
   };
   const UpdateConsts uc = update_consts_raw(a.lr, a.wd, a.factor[mat], gd.c, kScaleNone);
+
+  const bool vec = !md.transposed && (m & 3) == 0 &&
+                   ((reinterpret_cast<uintptr_t>(md.W) | reinterpret_cast<uintptr_t>(md.O)) & 15) == 0;
+  if (vec) {
+    // thread -> columns c4 .. c4 + 3, rows r0 + 8 k; ldc is a multiple of 8,
+    // so the four iterate elements are one 8-byte piece per bf16 part
+    static_assert(kEwCols == 128 && kEwRows == 64, "32 lanes x 4 columns, 8 warps x 8 rows");
+    const int c4 = (tid & 31) * 4;
+    const int r0 = tid >> 5;
+    const int64_t col = col0 + c4;
+    const bool col_ok = col < m;  // m % 4 == 0: all four columns are in range
+#pragma unroll
+    for (int ph = 0; ph < 2; ++ph) {
+      float4 w4[4], o4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t row = row0 + r0 + 8 * (4 * ph + j);
+        w4[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        o4[j] = w4[j];
+        if (!col_ok || row >= n) continue;
+        const int64_t k = row * ldc + col;
+        if (a.split) {
+          const uint2 hr = *reinterpret_cast<const uint2*>(oh + k);
+          const uint2 lr = *reinterpret_cast<const uint2*>(ol + k);
+          const float2 h0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hr.x));
+          const float2 h1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hr.y));
+          const float2 l0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lr.x));
+          const float2 l1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lr.y));
+          o4[j] = make_float4(h0.x + l0.x, h0.y + l0.y, h1.x + l1.x, h1.y + l1.y);
+        } else {
+          o4[j] = *reinterpret_cast<const float4*>(of + k);
+        }
+        if (md.W) w4[j] = *reinterpret_cast<const float4*>(md.W + row * m + col);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t row = row0 + r0 + 8 * (4 * ph + j);
+        if (!col_ok || row >= n) continue;
+        if (md.O) *reinterpret_cast<float4*>(md.O + row * m + col) = o4[j];
+        if (md.W) {
+          float4 w = w4[j];
+          w.x = fmaf(w.x, uc.keep, -uc.step * o4[j].x);
+          w.y = fmaf(w.y, uc.keep, -uc.step * o4[j].y);
+          w.z = fmaf(w.z, uc.keep, -uc.step * o4[j].z);
+          w.w = fmaf(w.w, uc.keep, -uc.step * o4[j].w);
+          *reinterpret_cast<float4*>(md.W + row * m + col) = w;
+        }
+      }
+    }
+    return;
+  }
 
   if (md.transposed) {
     // O'(caller i, j) is iterate element (j, i): read iterate rows j, two
