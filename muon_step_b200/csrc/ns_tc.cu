@@ -730,8 +730,10 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
       ok = false;
     }
     if (ok) {
-      ptx::bulk_wait_read<0>();  // the previous tile's stores have read every slot
-      for (int ch = ch_begin; ch < ch_begin + D; ++ch)
+      // the previous tile's stores have read every slot: fill them all, so
+      // that the first chunks' inputs travel while the accumulator is awaited
+      ptx::bulk_wait_read<0>();
+      for (int ch = ch_begin; ch < ch_begin + S; ++ch)
         if (live_chunk(ch)) issue_load(ch);
     }
   }
@@ -752,7 +754,7 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
     if (lane == 0) {
       // the load D chunks ahead reuses the slot of chunk ch + D - S, whose
       // stores are older than the newest kReuseWait groups
-      if (kInput && live_chunk(ch + D)) {
+      if (kInput && ch + D >= ch_begin + S && live_chunk(ch + D)) {
         ptx::bulk_wait_read<kReuseWait>();
         issue_load(ch + D);
       }
