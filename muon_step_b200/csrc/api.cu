@@ -542,7 +542,9 @@ muon_status_t upload(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
           encode_bf16_3d(&m[kTmXb0E], base + gd.xb_off[0], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
           encode_bf16_3d(&m[kTmXb1E], base + gd.xb_off[1], gd.c, gd.r, gd.ldc, gd.count, 32, 32, SW64) &&
           encode_bf16_3d(&m[kTmAE], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64) &&
-          encode_bf16_3d(&m[kTmBE], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64);
+          encode_bf16_3d(&m[kTmBE], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 32, 32, SW64) &&
+          encode_bf16_3d(&m[kTmAMN], base + gd.a_off, gd.r, gd.r, gd.ldr, gd.count, 64, 64, SW128) &&
+          encode_bf16_3d(&m[kTmBMN], base + gd.b_off, gd.r, gd.r, gd.ldr, gd.count, 64, 64, SW128);
       if (!ok) return MUON_ERR_CUDA;
     }
     auto* mmaps = reinterpret_cast<CUtensorMap*>(p->blob.data() + p->off_mat_tmaps);

@@ -64,7 +64,9 @@ enum TmapSlot : int {
   kTmXb1E = 8,   // bf16 iterate buffer 1, 64-byte swizzle
   kTmAE = 9,     // A, 64-byte swizzle
   kTmBE = 10,    // B, 64-byte swizzle
-  kTmPerGroup = 11
+  kTmAMN = 11,   // A, box {64, 64}: MN-major operand (a K block above the diagonal, read transposed)
+  kTmBMN = 12,   // B, box {64, 64}
+  kTmPerGroup = 13
 };
 
 struct GroupDesc {

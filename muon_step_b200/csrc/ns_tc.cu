@@ -36,13 +36,16 @@
 // a X + (b A + c A^2) X with A = X X^T):
 //
 //   Gram       A = X X^T. Symmetric: only pair tiles on or below the diagonal
-//              run; each 128 x 128 block on or below the diagonal is stored
-//              and, below the diagonal, mirrored. Step one folds s^2
+//              run, and only they are stored (the lower triangle of 256-row
+//              blocks, diagonal blocks in full). Step one folds s^2
 //              (X_0 = s N).
-//   Poly       B = b A + c A A^T (A symmetric), same tiling as Gram.
-//   Apply      X' = a X + B X: B is the K-major left operand, the iterate's
-//              high part the MN-major right operand (row-major X read as
-//              K x N); the epilogue adds a (high + low). Step one folds s.
+//   Poly       B = b A + c A A^T (A symmetric), same tiling and storage as
+//              Gram. A K block of A above its row block's diagonal is read
+//              from the transposed, stored position as an MN-major operand.
+//   Apply      X' = a X + B X: B is the left operand (K-major, or MN-major
+//              above the diagonal as in Poly), the iterate's high part the
+//              MN-major right operand (row-major X read as K x N); the
+//              epilogue adds a (high + low). Step one folds s.
 //   ApplyLast  the last step's Apply: O' = a X + B X, then the update of
 //              "Muon 优化器完全拆解…", Algorithm 1 steps four and five,
 //              W <- W (1 - lr wd) - lr gamma sqrt(max(n, m)) O', in the
@@ -103,8 +106,8 @@ constexpr int kTmapBytes = 128;
 constexpr int kTileQ = 4;  // chained launch: tile indices published ahead of their use
 
 // Facts of a tile kind that do not depend on the launch layout. Slot use:
-//   Gram       [bf16 out | bf16 mirror out]                            4 KB
-//   Poly       [bf16 A in, then mirror out | bf16 out]                 4 KB
+//   Gram       [bf16 out | unused]                                     4 KB
+//   Poly       [bf16 A in | bf16 out]                                  4 KB
 //   Apply      [bf16 iterate high in / out | bf16 low in / out]        4 KB
 //   ApplyLast  [bf16 high in | bf16 low in, then fp32 O out | fp32 W in / out]  8 KB
 template <int KIND>
@@ -113,10 +116,8 @@ struct KindT {
   static constexpr int kTiles = kApplyLike ? kApply : KIND;  // which tile tables to walk
   static constexpr bool kInput = (KIND != kGram);            // the epilogue loads inputs
   static constexpr int kSlotUse = (KIND == kApplyLast) ? 2 * kEpiF32 : 2 * kEpiB16;
-  // symmetric kinds: where the direct and mirrored outputs sit in a slot
-  // (Poly's mirror takes the area of its A input once every lane has read it)
+  // symmetric kinds: where the output sits in a slot (Poly's A input takes the first area)
   static constexpr int kOffSymOut = (KIND == kPoly) ? kEpiB16 : 0;
-  static constexpr int kOffSymMirror = (KIND == kPoly) ? 0 : kEpiB16;
 };
 
 // Launch layout: ring depth, epilogue warps (one per TMEM lane quarter, or
@@ -161,8 +162,10 @@ constexpr int kOffLow = kEpiB16;   // low part of the iterate in Apply-like slot
 constexpr int kSumsqSlots = 8;     // sum-of-squares slots per CTA and tile (most epilogue warps)
 constexpr int kOffLastW = kEpiF32;
 
-constexpr uint32_t kIdescKK = ptx::idesc_bf16(kPairTile, kPairTile, 0, 0);   // both K-major
-constexpr uint32_t kIdescKMN = ptx::idesc_bf16(kPairTile, kPairTile, 0, 1);  // B MN-major
+// instruction descriptors by operand major-ness (A side, B side; 1 = MN-major)
+__device__ __forceinline__ uint32_t idesc_of(bool a_mn, bool b_mn) {
+  return ptx::idesc_bf16(kPairTile, kPairTile, a_mn ? 1 : 0, b_mn ? 1 : 0);
+}
 
 struct TileCoord {
   int g;
@@ -338,8 +341,8 @@ __device__ __forceinline__ void raise_abort(const StageArgs& a, const Smem& s) {
 // Gram / Poly: one warp's 32 x 32 chunk of a block on or below the diagonal.
 template <int KIND>
 __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p, const GroupDesc& gd,
-                                              const TileCoord& tc, int row0, int col0, bool mirror,
-                                              uint8_t* slot, const float (&v)[32], int lane) {
+                                              const TileCoord& tc, int row0, int col0, uint8_t* slot,
+                                              const float (&v)[32], int lane) {
   float out[32];
   if (KIND == kGram) {
     // step one folds s^2; later steps store the product as it is (s^2 = 1)
@@ -366,7 +369,6 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p
     }
   }
   uint8_t* st_direct = slot + KindT<KIND>::kOffSymOut;
-  uint8_t* st_mirror = slot + KindT<KIND>::kOffSymMirror;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     Bf16x8 pk;
@@ -374,23 +376,11 @@ __device__ __forceinline__ void epi_symmetric(const StageArgs& a, const StepP& p
     for (int h = 0; h < 4; ++h) pk.v[h] = __floats2bfloat162_rn(out[8 * q + 2 * h], out[8 * q + 2 * h + 1]);
     *reinterpret_cast<Bf16x8*>(st_direct + sw64_chunk(lane, q)) = pk;
   }
-  if (mirror) {
-    // transposed chunk: row e of the mirror holds column e of this chunk (for
-    // Poly in the A input's area: every lane has read its row of A first)
-    if (KIND == kPoly) __syncwarp();
-    __nv_bfloat16* m16 = reinterpret_cast<__nv_bfloat16*>(st_mirror);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int off = sw64_chunk(e, lane >> 3) + (lane & 7) * 2;
-      m16[off >> 1] = __float2bfloat16_rn(out[e]);
-    }
-  }
   ptx::fence_async_shared();
   __syncwarp();
   if (lane == 0) {
     const void* tm = tmap(a, tc.g, KIND == kGram ? kTmAE : kTmBE);
     ptx::tma_store_3d(tm, st_direct, col0, row0, static_cast<int>(tc.b));
-    if (mirror) ptx::tma_store_3d(tm, st_mirror, row0, col0, static_cast<int>(tc.b));
   }
 }
 
@@ -580,6 +570,27 @@ __device__ __forceinline__ void epi_apply_last(const StageArgs& a, const StepP& 
 
 // -------------------------------------------------------------- per-tile roles
 
+// A and B are stored as their lower triangle of 256-row blocks only (the
+// Gram and Poly tiles with J <= I, diagonal blocks in full). A K block of a
+// symmetric operand's row block `blk` at or below the diagonal (k0 / 256 <=
+// blk) is read K-major from the stored rows; one above it is read from its
+// transposed position, block (k0 / 256, blk), as an MN-major operand: the
+// same values, since the matrix is symmetric.
+__device__ __forceinline__ bool sym_mn(int k0, int blk) { return k0 / kPairTile > blk; }
+
+// One CTA's half (rows blk * 256 + rank * 128 ..) of a symmetric operand's K block k0.
+__device__ __forceinline__ void load_sym_half(uint8_t* dst, const void* tm_k, const void* tm_mn,
+                                              uint32_t bar, int blk, int k0, uint32_t rank, int bz) {
+  const int row = blk * kPairTile + static_cast<int>(rank) * kHalf;
+  if (sym_mn(k0, blk)) {
+#pragma unroll
+    for (int q = 0; q < kHalf / 64; ++q)
+      ptx::tma_load_3d_pair(dst + q * (64 * kBK * 2), tm_mn, bar, row + q * 64, k0, bz);
+  } else {
+    ptx::tma_load_3d_pair(dst, tm_k, bar, k0, row, bz);
+  }
+}
+
 // Producer (one thread per CTA): the operand loads of one tile into the ring.
 // Returns false when a wait gives up (the caller aborts the pair).
 template <int KIND, int STAGES>
@@ -596,19 +607,25 @@ __device__ __forceinline__ bool produce_tile(const StageArgs& a, const Smem& s, 
     if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], diag ? kPairTx / 2 : kPairTx);
     const int k0 = kb * kBK;
     if (K::kApplyLike) {
-      ptx::tma_load_3d_pair(sa, tmap(a, tc.g, kTmB), leader_full[stage], k0,
-                            tc.I * kPairTile + rank * kHalf, bz);
+      // B (symmetric) rows I, then the iterate's column block J (MN-major)
+      load_sym_half(sa, tmap(a, tc.g, kTmB), tmap(a, tc.g, kTmBMN), leader_full[stage], tc.I, k0, rank, bz);
       const void* tx = tmap(a, tc.g, xsrc ? kTmXb1MN : kTmXb0MN);
 #pragma unroll
       for (int q = 0; q < kHalf / 64; ++q)
         ptx::tma_load_3d_pair(sb + q * (64 * kBK * 2), tx, leader_full[stage],
                               tc.J * kPairTile + rank * kHalf + q * 64, k0, bz);
-    } else {
-      const void* tm = (KIND == kGram) ? tmap(a, tc.g, xsrc ? kTmXb1K : kTmXb0K) : tmap(a, tc.g, kTmA);
+    } else if (KIND == kGram) {
+      const void* tm = tmap(a, tc.g, xsrc ? kTmXb1K : kTmXb0K);
       ptx::tma_load_3d_pair(sa, tm, leader_full[stage], k0, tc.I * kPairTile + rank * kHalf, bz);
       // on a diagonal tile each CTA's right-operand half is its left-operand rows
       if (tc.I != tc.J)
         ptx::tma_load_3d_pair(sb, tm, leader_full[stage], k0, tc.J * kPairTile + rank * kHalf, bz);
+    } else {
+      // Poly: A (symmetric) rows I and rows J
+      const void* tk = tmap(a, tc.g, kTmA);
+      const void* tmn = tmap(a, tc.g, kTmAMN);
+      load_sym_half(sa, tk, tmn, leader_full[stage], tc.I, k0, rank, bz);
+      if (tc.I != tc.J) load_sym_half(sb, tk, tmn, leader_full[stage], tc.J, k0, rank, bz);
     }
     if (++stage == STAGES) {
       stage = 0;
@@ -624,7 +641,6 @@ __device__ __forceinline__ bool mma_tile(const Smem& s, const TileCoord& tc, uin
                                          uint32_t& stage, uint32_t& phase, uint32_t& acc,
                                          uint32_t& acc_phase, bool& issued, uint64_t limit) {
   using K = KindT<KIND>;
-  const uint32_t idesc = K::kApplyLike ? kIdescKMN : kIdescKK;
   if (!ptx::mbar_wait(&s.tempty[acc], acc_phase ^ 1, limit, s.abort_flag)) return false;
   ptx::tc_fence_after();
   const uint32_t d = tmem_base + acc * kPairTile;
@@ -633,11 +649,18 @@ __device__ __forceinline__ bool mma_tile(const Smem& s, const TileCoord& tc, uin
     ptx::tc_fence_after();
     const uint32_t sa = ptx::smem_u32(s.ring + stage * kStageBytes);
     const uint32_t sb = (!K::kApplyLike && tc.I == tc.J) ? sa : sa + kABytes;
+    // major-ness of each side for this K block (Gram: X, always K-major;
+    // Poly: A both sides; Apply: B, then the iterate MN-major)
+    const int k0 = kb * kBK;
+    const bool a_mn = KIND != kGram && sym_mn(k0, tc.I);
+    const bool b_mn = K::kApplyLike || (KIND == kPoly && sym_mn(k0, tc.J));
+    const uint32_t idesc = idesc_of(a_mn, b_mn);
 #pragma unroll
     for (int k = 0; k < kBK / 16; ++k) {
-      const uint64_t ad = ptx::desc_sw128(sa + k * 32, 16, 1024);
-      const uint64_t bd = K::kApplyLike ? ptx::desc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
-                                        : ptx::desc_sw128(sb + k * 32, 16, 1024);
+      const uint64_t ad = a_mn ? ptx::desc_sw128(sa + k * 16 * 128, 64 * kBK * 2, 1024)
+                               : ptx::desc_sw128(sa + k * 32, 16, 1024);
+      const uint64_t bd = b_mn ? ptx::desc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
+                               : ptx::desc_sw128(sb + k * 32, 16, 1024);
       ptx::umma_bf16_pair(d, ad, bd, idesc, (kb | k) != 0);
     }
     issued = true;
@@ -686,7 +709,6 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
   constexpr int kReuseWait = S - 1 - D;  // store groups that may still be pending
   const GroupDesc& gd = a.groups[tc.g];
   const int row0 = tc.I * kPairTile + static_cast<int>(rank) * kHalf + quarter * 32;
-  const int bi = (tc.I * kPairTile + static_cast<int>(rank) * kHalf) / kHalf;
   const int bz = static_cast<int>(tc.b);
   const int mat = gd.first_mat + bz;
   // Apply-like: the current iterate's high part (the operand buffer) and low part
@@ -776,8 +798,7 @@ __device__ __forceinline__ bool epilogue_tile(const StageArgs& a, const StepP& p
       } else if (KIND == kApplyLast) {
         epi_apply_last(a, p, gd, tc, row0, col0, slot, v, lane, ssq);
       } else {
-        const int bj = col0 / kHalf;
-        if (bj <= bi) epi_symmetric<KIND>(a, p, gd, tc, row0, col0, bj < bi, slot, v, lane);
+        epi_symmetric<KIND>(a, p, gd, tc, row0, col0, slot, v, lane);
       }
     }
     // one bulk group per chunk (possibly empty), so "all but the newest
@@ -1043,6 +1064,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ChainL::kThreads, 1)
         if (ct.stage >= a.chain_stages) continue;
         const ChainPos cp = chain_pos(a, ct);
         if (cp.kind == kApply) r = mma_tile<kApply, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
+        else if (cp.kind == kPoly) r = mma_tile<kPoly, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
         else r = mma_tile<kGram, L::kStages>(s, cp.tc, tmem_base, stage, phase, acc, acc_phase, issued, limit);
       }
       if (!r) {

@@ -133,7 +133,7 @@ def expected_workspace(shapes, prec):
     ew = sum(math.ceil(n / 64) * math.ceil(m / 128) for n, m in shapes)
     off = al(ng * 160, 256)          # GroupDesc is 160 bytes
     off = al(off + nm * 88, 256)     # MatDesc is 88 bytes
-    off = al(off + (ng * 11 * 128 if prec == MUON_NS_BF16 else 0), 256)
+    off = al(off + (ng * 13 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + (nm * 2 * 128 if prec == MUON_NS_BF16 else 0), 256)
     off = al(off + ew * 4, 256)     # matrix of each elementwise tile
     tc = prec == MUON_NS_BF16

@@ -9,7 +9,8 @@ box coordinates and element accesses:
   (tiles per matrix, prefix bases per group), the tile decode (lower-triangle
   pair tiles for Gram and Poly, row-block-fastest tiles for Apply), the
   producer's operand loads, and the epilogue warps' 32 x 32 chunks with their
-  TMA loads and stores (direct and mirrored for the symmetric stages, the
+  TMA loads and stores (the symmetric stages' outputs in the lower
+  triangle of 256-row blocks, their operands read MN-major above it, the
   caller's W and O in its own orientation for the last step);
 * ``ns_small_kernel``, ``ns_mid_kernel`` and ``ns_tiny_kernel``: which
   thread touches which element of the iterate, the shared-memory tiles and
@@ -155,24 +156,40 @@ def run_stage(shapes, kind, npairs, wide):
             r, c, count, members = groups[g]
             assert I < cdiv(r, PAIR) and J <= (cdiv(c, PAIR) - 1 if table == APPLY else I)
             for rank in range(2):
-                # producer: operand loads (zero-filled past the extent)
+                # producer: operand loads (zero-filled past the extent); a
+                # symmetric operand's K block above the diagonal block is
+                # read MN-major from its transposed, stored position
+                def sym_half(blk, k0):
+                    row = blk * PAIR + rank * HALF
+                    if k0 // PAIR > blk:
+                        assert k0 // PAIR >= blk  # block (k0 / 256, blk) is in the stored triangle
+                        for q in range(HALF // 64):
+                            out.check_box(row + q * 64, k0, b, count, 2, store=False)
+                        return ("mn", k0 // PAIR, blk)
+                    out.check_box(k0, row, b, count, 2, store=False)
+                    return ("k", blk, k0 // PAIR)
+
                 for kb in range(kblocks):
                     k0 = kb * BK
                     if table == APPLY:
-                        out.check_box(k0, I * PAIR + rank * HALF, b, count, 2, store=False)
+                        src = sym_half(I, k0)
+                        assert src[1] >= src[2]  # only stored (lower-triangle) blocks of B are read
                         for q in range(HALF // 64):
                             out.check_box(J * PAIR + rank * HALF + q * 64, k0, b, count, 2, store=False)
-                    else:
+                    elif kind == GRAM:
                         out.check_box(k0, I * PAIR + rank * HALF, b, count, 2, store=False)
                         if I != J:
                             out.check_box(k0, J * PAIR + rank * HALF, b, count, 2, store=False)
+                    else:
+                        for blk in ((I,) if I == J else (I, J)):
+                            src = sym_half(blk, k0)
+                            assert src[1] >= src[2]  # only stored (lower-triangle) blocks of A
                 # epilogue warps
                 for ew in range(epi_warps):
                     quarter = (ew + 2) & 3
                     ch_begin = (ew // 4) * chunks_per_warp
                     row0 = I * PAIR + rank * HALF + quarter * 32
                     limit_c = c if table == APPLY else r
-                    bi = (I * PAIR + rank * HALF) // HALF
                     for ch in range(ch_begin, ch_begin + chunks_per_warp):
                         col0 = J * PAIR + ch * 32
                         if not (row0 < r and col0 < limit_c):
@@ -181,11 +198,8 @@ def run_stage(shapes, kind, npairs, wide):
                             name = "A" if kind == GRAM else "B"
                             if kind == POLY:
                                 out.check_box(col0, row0, b, count, 2, store=False)
-                            bj = col0 // HALF
-                            if bj <= bi:
-                                out.store(name, g, b, col0, row0, (32, 32), r, r)
-                                if bj < bi:
-                                    out.store(name, g, b, row0, col0, (32, 32), r, r)
+                            # the tile's own chunk only: the stored lower triangle
+                            out.store(name, g, b, col0, row0, (32, 32), r, r)
                         else:
                             out.check_box(col0, row0, b, count, 2, store=False)  # high part in
                             if kind == APPLY:
@@ -211,9 +225,10 @@ SHAPE_SETS = [
 @pytest.mark.parametrize("npairs", [74, 5])
 @pytest.mark.parametrize("wide", [False, True])
 def test_symmetric_stages_write_every_element_once(shapes, npairs, wide):
-    """Gram and Poly store every element of A and B exactly once: the direct
-    stores cover the 128 x 128 blocks on and below the diagonal, the mirrored
-    stores those above it."""
+    """Gram and Poly store every element of the lower triangle of 256-row
+    blocks of A and B (diagonal blocks in full) exactly once and nothing
+    above it; the consumers read the blocks above from their transposed
+    positions."""
     for kind, name in ((GRAM, "A"), (POLY, "B")):
         groups, out = run_stage(shapes, kind, npairs, wide)
         for g, (r, c, count, _) in enumerate(groups):
@@ -222,7 +237,10 @@ def test_symmetric_stages_write_every_element_once(shapes, npairs, wide):
                 continue
             w = out.writes[(name, g)]
             assert w.shape == (count, r, r)
-            assert (w == 1).all(), (name, r, c, np.unique(w))
+            blk = np.arange(r) // PAIR
+            lower = blk[:, None] >= blk[None, :]
+            assert (w[:, lower] == 1).all(), (name, r, c, np.unique(w[:, lower]))
+            assert (w[:, ~lower] == 0).all(), (name, r, c)
 
 
 @pytest.mark.parametrize("shapes", SHAPE_SETS)
